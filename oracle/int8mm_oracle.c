@@ -1,0 +1,339 @@
+/*
+ * Plain CPU oracle for the LLM.int8() matrix multiplication  Y = X * W.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the slow, obviously-correct
+ * statement of what the GPU library computes.  Only the test suite, the
+ * package smoke check and the benchmark's CPU-baseline leg may load it.  It
+ * shares no code, header, table or constant generator with the CUDA path.
+ *
+ * Source of the method: "LLM.int8(): 8-bit Matrix Multiplication for
+ * Transformers at Scale" (Dettmers, Lewis, Belkada, Zettlemoyer, 2022),
+ * abstract: a two-part procedure for the feed-forward and attention
+ * projection matmuls -- vector-wise quantisation with one normalisation
+ * constant per inner-product vector, plus a mixed-precision decomposition
+ * that moves the outlier feature dimensions into a 16-bit matmul.  The axolotl
+ * "llama3-model-quantization" summary of the same talk adds: outliers sit in
+ * specific feature columns of the input ("Understanding Outliers in
+ * Transformer Models"), they are processed in 16 bit and the rest in 8 bit
+ * ("Key Points"), and quantisation normalises by the maximum value
+ * ("Key Points", block-wise paragraph).  The scite report for nuQmm quotes
+ * that LLM.int8() rounds to the nearest quantisation level (RTN).
+ *
+ * Numerics (the plainest reading where the pages leave a step open):
+ *   - fp16 inputs are converted to fp32 exactly;
+ *   - a feature column k is an outlier when |X[m,k]| >= threshold for ANY
+ *     row m of this call; the outlier list is ascending;
+ *   - row absmax ra[m] is taken over the non-outlier columns only;
+ *   - scale = 127.0f / absmax (IEEE fp32 division, round to nearest even),
+ *     q = round-half-even(x * scale) in fp32, clamped to [-127, 127];
+ *     absmax == 0 gives q = 0 and a stored absmax of 0;
+ *   - weight absmax ca[n] is taken per output channel over ALL K;
+ *   - int8 products are summed exactly (int64, then checked to fit int32);
+ *   - the 16-bit outlier product sums fp32(xo)*fp32(wo) in fp32 in
+ *     ascending outlier order;
+ *   - outlier weight rows come from the fp16 rows kept at preparation time,
+ *     else from the dequantised int8 row fp16(q * ca / 127);
+ *   - y = fp16( (float)acc * ra[m] * ca[n] / 16129 + o ), left to right.
+ *
+ * Build: gcc -O2 -ffp-contract=off (no fast-math), -pthread.
+ */
+#include <fenv.h>
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* IEEE binary16 <-> binary32, written from the format definition.          */
+/* ------------------------------------------------------------------------ */
+
+float orc_half_to_float(uint16_t h) {
+    int sign = (h >> 15) & 1;
+    int exp = (h >> 10) & 0x1f;
+    int mant = h & 0x3ff;
+    float v;
+    if (exp == 0) {
+        v = ldexpf((float)mant, -24); /* zero or subnormal: mant * 2^-24 */
+    } else if (exp == 31) {
+        v = mant ? NAN : INFINITY;
+    } else {
+        v = ldexpf((float)(1024 + mant), exp - 25); /* (1.mant) * 2^(exp-15) */
+    }
+    return sign ? -v : v;
+}
+
+/* Round-to-nearest-even conversion of a binary32 value to binary16 bits. */
+uint16_t orc_float_to_half(float f) {
+    uint16_t sign = signbit(f) ? 0x8000u : 0u;
+    if (isnan(f)) return (uint16_t)(sign | 0x7e00u);
+    float a = fabsf(f);
+    /* 65520 is the midpoint between 65504 (odd mantissa) and 2^16: ties go
+       to the even neighbour, which overflows to infinity. */
+    if (a >= 65520.0f) return (uint16_t)(sign | 0x7c00u);
+    if (a < ldexpf(1.0f, -14)) {
+        /* subnormal range: value = n * 2^-24, n rounded half-even; n == 1024
+           lands exactly on the smallest normal, whose bits are 0x0400. */
+        float n = nearbyintf(ldexpf(a, 24));
+        return (uint16_t)(sign | (uint16_t)n);
+    }
+    int e;
+    frexpf(a, &e);          /* a = fr * 2^e, fr in [0.5, 1) */
+    e -= 1;                 /* a = 1.x * 2^e */
+    float m = nearbyintf(ldexpf(a, 10 - e)); /* in [1024, 2048] */
+    if (m == 2048.0f) {
+        m = 1024.0f;
+        e += 1;
+    }
+    if (e + 15 >= 31) return (uint16_t)(sign | 0x7c00u);
+    return (uint16_t)(sign | (uint16_t)((e + 15) << 10) | (uint16_t)((int)m - 1024));
+}
+
+/* ------------------------------------------------------------------------ */
+/* Shared quantisation rule: one vector, its absmax, scale and codes.        */
+/* ------------------------------------------------------------------------ */
+
+static int8_t quantize_one(float x, float scale) {
+    float r = nearbyintf(x * scale); /* fp32 product, then half-even */
+    if (r > 127.0f) r = 127.0f;
+    if (r < -127.0f) r = -127.0f;
+    return (int8_t)r;
+}
+
+/* ------------------------------------------------------------------------ */
+/* (a) Outlier feature detection.                                            */
+/* A column is an outlier when any row reaches the threshold in magnitude.   */
+/* Writes the ascending outlier column list to idx (capacity K) and returns  */
+/* its length.                                                               */
+/* ------------------------------------------------------------------------ */
+
+int orc_detect_outliers(const uint16_t* X, int M, int K, float thr, int32_t* idx) {
+    fesetround(FE_TONEAREST);
+    int n = 0;
+    for (int k = 0; k < K; ++k) {
+        int flag = 0;
+        for (int m = 0; m < M; ++m) {
+            float x = orc_half_to_float(X[(size_t)m * K + k]);
+            if (fabsf(x) >= thr) {
+                flag = 1;
+                break;
+            }
+        }
+        if (flag) idx[n++] = k;
+    }
+    return n;
+}
+
+/* ------------------------------------------------------------------------ */
+/* (b) Row-wise (vector-wise) int8 quantisation of X with the outlier        */
+/* columns removed, plus the fp16 outlier sub-matrix Xo (M x n_o).           */
+/* ------------------------------------------------------------------------ */
+
+void orc_quantize_rows(const uint16_t* X, int M, int K, const int32_t* idx, int n_o,
+                       int8_t* Xq, float* ra, uint16_t* Xo) {
+    fesetround(FE_TONEAREST);
+    unsigned char* is_out = (unsigned char*)calloc((size_t)K > 0 ? (size_t)K : 1, 1);
+    for (int j = 0; j < n_o; ++j) is_out[idx[j]] = 1;
+    for (int m = 0; m < M; ++m) {
+        const uint16_t* row = X + (size_t)m * K;
+        float amax = 0.0f;
+        for (int k = 0; k < K; ++k) {
+            if (is_out[k]) continue;
+            float a = fabsf(orc_half_to_float(row[k]));
+            if (a > amax) amax = a;
+        }
+        ra[m] = amax;
+        float scale = amax > 0.0f ? 127.0f / amax : 0.0f;
+        for (int k = 0; k < K; ++k) {
+            int8_t q = 0;
+            if (!is_out[k] && amax > 0.0f) q = quantize_one(orc_half_to_float(row[k]), scale);
+            Xq[(size_t)m * K + k] = q;
+        }
+        for (int j = 0; j < n_o; ++j) Xo[(size_t)m * n_o + j] = row[idx[j]];
+    }
+    free(is_out);
+}
+
+/* ------------------------------------------------------------------------ */
+/* (c) One-time per-output-channel int8 quantisation of W (K x N, row-major) */
+/* into Wq (N x K: row n holds output channel n) and ca (N).                 */
+/* ------------------------------------------------------------------------ */
+
+void orc_quantize_weight(const uint16_t* W, int K, int N, int8_t* Wq, float* ca) {
+    fesetround(FE_TONEAREST);
+    for (int n = 0; n < N; ++n) {
+        float amax = 0.0f;
+        for (int k = 0; k < K; ++k) {
+            float a = fabsf(orc_half_to_float(W[(size_t)k * N + n]));
+            if (a > amax) amax = a;
+        }
+        ca[n] = amax;
+        float scale = amax > 0.0f ? 127.0f / amax : 0.0f;
+        for (int k = 0; k < K; ++k) {
+            int8_t q = 0;
+            if (amax > 0.0f) q = quantize_one(orc_half_to_float(W[(size_t)k * N + n]), scale);
+            Wq[(size_t)n * K + k] = q;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* (d1) Exact int8 product acc[m,n] = sum_k Xq[m,k] * Wq[n,k].               */
+/* Rows are split across threads; each sum is an exact int64 checked to fit */
+/* int32.  Returns 0, or -1 if some sum does not fit.                        */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    const int8_t* Xq;
+    const int8_t* Wq;
+    int M, N, K, m0, m1;
+    int32_t* acc;
+    int overflow;
+} gemm_job;
+
+static void* gemm_rows(void* p) {
+    gemm_job* j = (gemm_job*)p;
+    for (int m = j->m0; m < j->m1; ++m) {
+        const int8_t* a = j->Xq + (size_t)m * j->K;
+        for (int n = 0; n < j->N; ++n) {
+            const int8_t* b = j->Wq + (size_t)n * j->K;
+            int64_t s = 0;
+            for (int k = 0; k < j->K; ++k) s += (int64_t)a[k] * (int64_t)b[k];
+            if (s > INT32_MAX || s < INT32_MIN) j->overflow = 1;
+            j->acc[(size_t)m * j->N + n] = (int32_t)s;
+        }
+    }
+    return NULL;
+}
+
+int orc_int8_gemm(const int8_t* Xq, const int8_t* Wq, int M, int N, int K, int32_t* acc,
+                  int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > M) nthreads = M > 0 ? M : 1;
+    gemm_job* jobs = (gemm_job*)calloc((size_t)nthreads, sizeof(gemm_job));
+    pthread_t* th = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t].Xq = Xq;
+        jobs[t].Wq = Wq;
+        jobs[t].M = M;
+        jobs[t].N = N;
+        jobs[t].K = K;
+        jobs[t].m0 = (int)((int64_t)M * t / nthreads);
+        jobs[t].m1 = (int)((int64_t)M * (t + 1) / nthreads);
+        jobs[t].acc = acc;
+        jobs[t].overflow = 0;
+        if (t > 0) pthread_create(&th[t], NULL, gemm_rows, &jobs[t]);
+    }
+    if (nthreads > 0) gemm_rows(&jobs[0]);
+    int overflow = jobs[0].overflow;
+    for (int t = 1; t < nthreads; ++t) {
+        pthread_join(th[t], NULL);
+        overflow |= jobs[t].overflow;
+    }
+    free(jobs);
+    free(th);
+    return overflow ? -1 : 0;
+}
+
+/* The same exact sum at a list of (m, n) points only. */
+int orc_int8_gemm_points(const int8_t* Xq, const int8_t* Wq, int K, const int32_t* pm,
+                         const int32_t* pn, int npts, int32_t* acc) {
+    int overflow = 0;
+    for (int p = 0; p < npts; ++p) {
+        const int8_t* a = Xq + (size_t)pm[p] * K;
+        const int8_t* b = Wq + (size_t)pn[p] * K;
+        int64_t s = 0;
+        for (int k = 0; k < K; ++k) s += (int64_t)a[k] * (int64_t)b[k];
+        if (s > INT32_MAX || s < INT32_MIN) overflow = 1;
+        acc[p] = (int32_t)s;
+    }
+    return overflow ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* The fp16 weight rows of the outlier dimensions.                           */
+/* Wo (n_o x N): row j is W[idx[j], :] -- the fp16 row kept at preparation   */
+/* time when idx[j] is among keep_idx, else the dequantised row              */
+/* fp16((float)Wq[n, idx[j]] * ca[n] / 127).                                 */
+/* W_keep is n_keep x N, row i holding W[keep_idx[i], :].                    */
+/* ------------------------------------------------------------------------ */
+
+void orc_gather_w_outlier(const uint16_t* W_keep, const int32_t* keep_idx, int n_keep,
+                          const int8_t* Wq, const float* ca, int K, int N, const int32_t* idx,
+                          int n_o, uint16_t* Wo) {
+    fesetround(FE_TONEAREST);
+    for (int j = 0; j < n_o; ++j) {
+        int k = idx[j];
+        int slot = -1;
+        for (int i = 0; i < n_keep; ++i)
+            if (keep_idx[i] == k) {
+                slot = i;
+                break;
+            }
+        for (int n = 0; n < N; ++n) {
+            uint16_t w;
+            if (slot >= 0) {
+                w = W_keep[(size_t)slot * N + n];
+            } else {
+                float t = (float)Wq[(size_t)n * K + k] * ca[n];
+                w = orc_float_to_half(t / 127.0f);
+            }
+            Wo[(size_t)j * N + n] = w;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* (d2) 16-bit outlier product o[m,n] = sum_j Xo[m,j] * Wo[j,n] in fp32,     */
+/* ascending j.                                                              */
+/* ------------------------------------------------------------------------ */
+
+static float outlier_dot(const uint16_t* Xo, const uint16_t* Wo, int N, int n_o, int m, int n) {
+    float s = 0.0f;
+    for (int j = 0; j < n_o; ++j)
+        s += orc_half_to_float(Xo[(size_t)m * n_o + j]) * orc_half_to_float(Wo[(size_t)j * N + n]);
+    return s;
+}
+
+void orc_outlier_gemm(const uint16_t* Xo, const uint16_t* Wo, int M, int N, int n_o, float* o) {
+    fesetround(FE_TONEAREST);
+    for (int m = 0; m < M; ++m)
+        for (int n = 0; n < N; ++n) o[(size_t)m * N + n] = outlier_dot(Xo, Wo, N, n_o, m, n);
+}
+
+/* ------------------------------------------------------------------------ */
+/* (d3) Dequantise and combine: y = fp16(acc * ra * ca / 16129 + o).         */
+/* ------------------------------------------------------------------------ */
+
+static uint16_t combine(int32_t acc, float ra, float ca, float o) {
+    float v = (float)acc;
+    v = v * ra;
+    v = v * ca;
+    v = v / 16129.0f;
+    v = v + o;
+    return orc_float_to_half(v);
+}
+
+void orc_epilogue(const int32_t* acc, const float* ra, const float* ca, const float* o, int M,
+                  int N, uint16_t* Y) {
+    fesetround(FE_TONEAREST);
+    for (int m = 0; m < M; ++m)
+        for (int n = 0; n < N; ++n) {
+            size_t i = (size_t)m * N + n;
+            Y[i] = combine(acc[i], ra[m], ca[n], o ? o[i] : 0.0f);
+        }
+}
+
+/* y at a list of points, from the quantised operands (acc computed here). */
+int orc_forward_points(const int8_t* Xq, const float* ra, const int8_t* Wq, const float* ca,
+                       const uint16_t* Xo, const uint16_t* Wo, int K, int N, int n_o,
+                       const int32_t* pm, const int32_t* pn, int npts, int32_t* acc_out,
+                       uint16_t* y_out) {
+    fesetround(FE_TONEAREST);
+    int rc = orc_int8_gemm_points(Xq, Wq, K, pm, pn, npts, acc_out);
+    for (int p = 0; p < npts; ++p) {
+        float o = outlier_dot(Xo, Wo, N, n_o, pm[p], pn[p]);
+        y_out[p] = combine(acc_out[p], ra[pm[p]], ca[pn[p]], o);
+    }
+    return rc;
+}

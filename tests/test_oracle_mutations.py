@@ -1,0 +1,79 @@
+"""Pin strength: plant plausible mistakes in copies of the oracle source and
+check that the pins catch every one.  The mistakes live only in temporary
+copies compiled on the CPU; the committed oracle is never changed."""
+from __future__ import annotations
+
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+MUTATIONS = {
+    "threshold_strict": ("if (fabsf(x) >= thr)", "if (fabsf(x) > thr)"),
+    "outliers_in_row_absmax": ("if (is_out[k]) continue;", ";"),
+    "outlier_column_not_zeroed": ("if (!is_out[k] && amax > 0.0f)", "if (amax > 0.0f)"),
+    "round_half_away": ("float r = nearbyintf(x * scale);", "float r = roundf(x * scale);"),
+    "divide_instead_of_scale": ("float r = nearbyintf(x * scale);", "float r = nearbyintf(x / (1.0f / scale));"),
+    "clamp_to_126": ("if (r > 127.0f) r = 127.0f;", "if (r > 126.0f) r = 126.0f;"),
+    "weight_transposed": ("float a = fabsf(orc_half_to_float(W[(size_t)k * N + n]));",
+                          "float a = fabsf(orc_half_to_float(W[(size_t)(k % N) * N + (n % K)]));"),
+    "weight_absmax_skips_row0": ("for (int k = 0; k < K; ++k) {\n            float a = fabsf(orc_half_to_float(W[",
+                                 "for (int k = 1; k < K; ++k) {\n            float a = fabsf(orc_half_to_float(W["),
+    "gemm_drops_last_k": ("for (int k = 0; k < j->K; ++k) s +=", "for (int k = 0; k + 1 < j->K; ++k) s +="),
+    "outlier_term_dropped": ("v = v + o;", "v = v + 0.0f * o;"),
+    "outlier_sign": ("v = v + o;", "v = v - o;"),
+    "wrong_denominator": ("v = v / 16129.0f;", "v = v / 16384.0f;"),
+    "kept_row_ignored": ("if (slot >= 0) {\n                w = W_keep", "if (slot >= 1000000) {\n                w = W_keep"),
+    "xo_wrong_column": ("Xo[(size_t)m * n_o + j] = row[idx[j]];", "Xo[(size_t)m * n_o + j] = row[idx[j] > 0 ? idx[j] - 1 : 0];"),
+}
+
+
+def _pin_suite():
+    """Run a fast subset of the pins; return the names of those that fail."""
+    failed = []
+    checks = {
+        "worked_example": pins.test_worked_example_golden,
+        "threshold_equality": pins.test_value_exactly_at_threshold_is_outlier,
+        "absmax_127": pins.test_absmax_maps_to_127,
+        "lossless": pins.test_lossless_integer_inputs,
+        "all_outlier": pins.test_all_outlier_reduces_to_fp16_matmul,
+        "error_bound": pins.test_result_within_method_error_bound,
+        "dequantised_rows": pins.test_dequantised_outlier_rows_when_not_kept,
+    }
+    for amax in (5.99609375, 3.140625, 40.96875, 0.46044921875, 1.5947265625):
+        checks[f"rule_exhaustive_{amax}"] = (lambda a=amax: pins.test_quantisation_rule_exhaustive(a))
+    for seed in range(40):
+        checks[f"brute_force_{seed}"] = (lambda s=seed: pins.test_brute_force_tiny(s))
+    for name, fn in checks.items():
+        try:
+            fn()
+        except Exception:  # noqa: BLE001 - any failure counts as caught
+            failed.append(name)
+    return failed
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, tmp_path):
+    old, new = MUTATIONS[name]
+    with open(oracle._SRC) as f:
+        src = f.read()
+    assert src.count(old) >= 1, f"mutation anchor for {name} not found"
+    mutated = src.replace(old, new, 1)
+    c_path = os.path.join(tmp_path, "mut.c")
+    so_path = os.path.join(tmp_path, "libmut.so")
+    with open(c_path, "w") as f:
+        f.write(mutated)
+    subprocess.run(["gcc", *oracle._CFLAGS, "-o", so_path, c_path, "-lm"], check=True)
+    oracle._swap_library(so_path)
+    try:
+        failed = _pin_suite()
+    finally:
+        oracle._swap_library(None)
+    assert failed, f"planted mistake {name!r} passed every pin"
+
+
+def test_unmutated_oracle_passes_suite():
+    assert _pin_suite() == []
