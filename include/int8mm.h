@@ -1,0 +1,182 @@
+/*
+ * int8mm -- the LLM.int8() matrix multiplication Y = X W on NVIDIA B200 (sm_100a).
+ *
+ * Method: "LLM.int8(): 8-bit Matrix Multiplication for Transformers at Scale"
+ * (Dettmers, Lewis, Belkada, Zettlemoyer, 2022), abstract: Int8 matmul for the
+ * feed-forward and attention-projection layers of a transformer, as a
+ * two-part procedure --
+ *   1. vector-wise quantisation: one normalisation constant per row of X and
+ *      one per output column of W ("separate normalization constants for each
+ *      inner product");
+ *   2. mixed-precision decomposition: the outlier feature dimensions of X go
+ *      to a 16-bit matmul, everything else is multiplied in 8 bit.
+ * Outliers are feature columns of the input batch (axolotl
+ * "llama3-model-quantization", "Understanding Outliers in Transformer
+ * Models"); quantisation normalises by the absolute maximum ("Key Points") and
+ * rounds to the nearest level (scite report for nuQmm, which quotes LLM.int8()
+ * as RTN); a 16/32-bit checkpoint is "converted to Int8" once at load
+ * (abstract) -- int8mm_prepare_weight.
+ *
+ * What one int8mm_forward computes (X: M x K, W: K x N, both fp16 row-major):
+ *   (a) O = ascending list of columns k with |X[m,k]| >= threshold for any m;
+ *   (b) ra[m] = max_{k not in O} |X[m,k]|,  Xq[m,k] = k in O ? 0 :
+ *       round_half_even(X[m,k] * (127.0f / ra[m])) clamped to [-127, 127]
+ *       (fp32 arithmetic, ra = 0 gives Xq = 0);
+ *   (c) (at prepare time) ca[n] = max_k |W[k,n]| over all k and
+ *       Wq[n,k] = round_half_even(W[k,n] * (127.0f / ca[n]));
+ *   (d) Y[m,n] = fp16( sum_k Xq[m,k] Wq[n,k] * ra[m] * ca[n] / 127^2
+ *                      + sum_{j} X[m,O[j]] * Wo[j,n] ),
+ *       the first sum exact in int32, the second in fp32; Wo[j,:] is the fp16
+ *       row W[O[j],:] when O[j] was kept at prepare time, else the dequantised
+ *       row fp16(Wq[n,O[j]] * ca[n] / 127).
+ *
+ * Conventions for every call:
+ *   - fp16 tensors are passed as pointers to IEEE binary16 bit patterns
+ *     (uint16_t); all matrices are row-major and densely packed.
+ *   - "device" pointers point to memory of the current CUDA device; the
+ *     caller allocates and owns all memory.  The library allocates nothing
+ *     on the device and keeps no global state between calls.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are stream-ordered and do not synchronise the host,
+ *     except where a function says so.
+ *   - Shape rules: M >= 1; K, N >= 16 and multiples of 16; K <= 131072
+ *     (so that K * 127^2 fits int32); M, N < 2^31.
+ *   - Alignment rules: X, W, Y 16-byte aligned; weight and workspace buffers
+ *     256-byte aligned.
+ *   - Argument errors are returned synchronously and leave every buffer
+ *     untouched.  Errors found on the device (a wait that ran out, more
+ *     outliers than the workspace holds) are recorded in the workspace and
+ *     read back with int8mm_get_device_status.
+ */
+#ifndef INT8MM_H
+#define INT8MM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    INT8MM_OK = 0,
+    INT8MM_ERR_INVALID_ARGUMENT = 1,   /* a shape, count or pointer breaks the rules above */
+    INT8MM_ERR_MISALIGNED = 2,         /* a pointer breaks the alignment rules */
+    INT8MM_ERR_WORKSPACE_TOO_SMALL = 3,/* buffer smaller than the matching *_bytes() */
+    INT8MM_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not compute capability 10.0 */
+    INT8MM_ERR_CUDA = 5,               /* a CUDA runtime / driver call failed */
+    INT8MM_ERR_TIMEOUT = 6,            /* (device) an in-kernel wait ran out; outputs invalid */
+    INT8MM_ERR_OUTLIER_OVERFLOW = 7    /* (device) more outlier columns than max_outliers; outputs invalid */
+} int8mm_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* int8mm_status_string(int8mm_status s);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int int8mm_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* Prepared (int8) weight -- "a 16/32-bit checkpoint can be loaded, converted */
+/* to Int8, and used immediately" (LLM.int8() abstract).                       */
+/* ------------------------------------------------------------------------ */
+
+/* Views into one caller-owned device buffer, filled by int8mm_prepare_weight.
+ * The buffer outlives every forward that uses the weight; W itself may be
+ * freed once int8mm_prepare_weight returns. */
+typedef struct {
+    int32_t K, N, n_keep;
+    int8_t* wq;          /* device, N x K int8: row n = output channel n, K contiguous */
+    float* col_absmax;   /* device, N: ca[n] = max_k |W[k,n]| */
+    uint16_t* w_keep;    /* device, n_keep x N fp16: row i = W[keep_idx[i], :] */
+    int32_t* keep_idx;   /* device, n_keep, strictly ascending column indices */
+    int32_t* keep_slot;  /* device, K: i if k == keep_idx[i], else -1 */
+} int8mm_weight;
+
+/* Bytes of the device buffer int8mm_prepare_weight needs. */
+size_t int8mm_weight_bytes(int K, int N, int n_keep);
+
+/* Convert W (device, K x N fp16) into the int8 weight.
+ *   keep_idx_host: host array of n_keep strictly ascending feature indices in
+ *     [0, K) whose fp16 rows W[k, :] are kept for the 16-bit outlier product
+ *     (the feature dimensions expected to carry outliers; NULL iff n_keep == 0).
+ *   buf / buf_bytes: device buffer of at least int8mm_weight_bytes(K, N, n_keep).
+ *   out: host struct receiving the views into buf.
+ * Synchronises `stream` before returning (it copies from host memory). */
+int8mm_status int8mm_prepare_weight(const uint16_t* W, int K, int N, const int32_t* keep_idx_host,
+                                    int n_keep, void* buf, size_t buf_bytes, int8mm_weight* out,
+                                    void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Forward  Y = X W                                                           */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of device workspace a forward with these sizes needs.  max_outliers
+ * (0 <= max_outliers <= K) bounds how many outlier columns one call may
+ * detect; K is always safe. */
+size_t int8mm_workspace_bytes(int M, int K, int N, int max_outliers);
+
+/* Zero-fill a workspace (stream-ordered).  Needed once before its first
+ * forward, and again after a forward that reported a device error; every
+ * successful forward leaves the workspace ready for the next one. */
+int8mm_status int8mm_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Y (device, M x N fp16) = the LLM.int8() product of X (device, M x K fp16)
+ * and the prepared weight w, with outlier threshold `threshold` (> 0, may be
+ * +inf to disable the decomposition).  ws is a zero-initialised workspace of
+ * at least int8mm_workspace_bytes(M, w->K, w->N, max_outliers) bytes; it
+ * must not be used by two forwards that overlap on the GPU. */
+int8mm_status int8mm_forward(const uint16_t* X, int M, const int8mm_weight* w, float threshold,
+                             int max_outliers, uint16_t* Y, void* ws, size_t ws_bytes,
+                             void* stream);
+
+enum {
+    INT8MM_PATH_AUTO = 0,    /* decode kernel for M <= 16, tiled GEMM otherwise */
+    INT8MM_PATH_GEMM = 1,    /* detect -> quantise -> gather -> tcgen05 GEMM, any M */
+    INT8MM_PATH_DECODE = 2   /* single fused weight-streaming kernel, M <= 16 */
+};
+
+typedef struct {
+    int path;                /* INT8MM_PATH_* */
+    int32_t* acc_out;        /* optional device M x N int32: the exact int8 sums (for tests) */
+    uint64_t wait_limit_ns;  /* bound on every in-kernel wait; 0 = 2 s */
+    void* main_start_event;  /* optional cudaEvent_t recorded on `stream` just before the main
+                                kernel (the tcgen05 GEMM or the fused decode kernel) ... */
+    void* main_stop_event;   /* ... and just after it; both or neither (for timing). */
+    uint32_t test_flags;     /* 0 in normal use.  INT8MM_TEST_WITHHOLD_SIGNAL: the main kernel never
+                                sends one internal "data ready" signal, so the wait for it runs
+                                out after wait_limit_ns and the call reports INT8MM_ERR_TIMEOUT
+                                (exercises the timeout path without faulting the GPU). */
+} int8mm_forward_opts;
+
+enum { INT8MM_TEST_WITHHOLD_SIGNAL = 1 };
+
+/* int8mm_forward with options (opts may be NULL = defaults). */
+int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w, float threshold,
+                                int max_outliers, uint16_t* Y, void* ws, size_t ws_bytes,
+                                const int8mm_forward_opts* opts, void* stream);
+
+/* Device pointers to the intermediates a forward leaves in its workspace. */
+typedef struct {
+    int32_t* status;       /* 1 word: bit 0 timeout, bit 1 outlier overflow */
+    int32_t* n_outliers;   /* 1 word: number of outlier columns detected (may exceed capacity) */
+    int32_t* outlier_idx;  /* K words: ascending outlier columns (first min(n, capacity) valid) */
+    float* row_absmax;     /* M: ra */
+    int8_t* xq;            /* M x K int8: Xq */
+    uint16_t* xo;          /* M x kp fp16: X[:, O] (GEMM path only), zero-padded */
+    int32_t kp;            /* row length of xo (max_outliers rounded up to 64) */
+} int8mm_workspace_view;
+
+int8mm_status int8mm_workspace_view_get(void* ws, size_t ws_bytes, int M, int K, int N,
+                                        int max_outliers, int8mm_workspace_view* out);
+
+/* Wait for `stream`, then report the device-side status of the last forward
+ * that used ws: INT8MM_OK, INT8MM_ERR_TIMEOUT or INT8MM_ERR_OUTLIER_OVERFLOW.
+ * If n_outliers is not NULL it receives the detected outlier count.
+ * Synchronises the host with `stream`. */
+int8mm_status int8mm_get_device_status(const void* ws, void* stream, int32_t* n_outliers);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INT8MM_H */

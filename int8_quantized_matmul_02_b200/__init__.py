@@ -1,0 +1,173 @@
+"""LLM.int8() matrix multiplication for NVIDIA B200 (sm_100a).
+
+Python face of ``libint8mm`` (C-ABI in ``include/int8mm.h``).  PyTorch is used
+for device memory and streams only; every step of the product runs in the
+library's CUDA kernels, and there is no CPU fallback.
+
+Method: "LLM.int8(): 8-bit Matrix Multiplication for Transformers at Scale"
+(Dettmers et al., 2022), abstract -- vector-wise int8 quantisation plus a
+16-bit matmul over the outlier feature dimensions, for the feed-forward and
+attention-projection layers of a transformer.
+
+    w  = prepare_weight(W_fp16_KxN, keep_idx)      # once, at load
+    ws = Workspace(M, K, N)                         # reusable scratch
+    Y  = forward(X_fp16_MxK, w, threshold=6.0, workspace=ws)
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import torch
+
+from . import _abi
+from ._abi import PATH_AUTO, PATH_DECODE, PATH_GEMM, Int8mmError
+
+__all__ = [
+    "PreparedWeight", "Workspace", "prepare_weight", "forward", "device_status", "library",
+    "Int8mmError", "PATH_AUTO", "PATH_GEMM", "PATH_DECODE",
+]
+
+_PATHS = {"auto": PATH_AUTO, "gemm": PATH_GEMM, "decode": PATH_DECODE}
+
+
+def library():
+    """The loaded ctypes handle of libint8mm.so (raises if it is missing)."""
+    return _abi.load()
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _view(buf: torch.Tensor, ptr: int, count: int, dtype: torch.dtype, shape=None) -> torch.Tensor:
+    off = int(ptr) - buf.data_ptr()
+    nbytes = count * torch.empty(0, dtype=dtype).element_size()
+    t = buf[off: off + nbytes].view(dtype)
+    return t.view(*shape) if shape is not None else t
+
+
+class PreparedWeight:
+    """An int8 weight in one device buffer (see ``int8mm_weight`` in the header)."""
+
+    def __init__(self, buf: torch.Tensor, st: _abi.Weight):
+        self.buf = buf
+        self.struct = st
+        self.K, self.N, self.n_keep = st.K, st.N, st.n_keep
+
+    @property
+    def wq(self) -> torch.Tensor:           # N x K int8
+        return _view(self.buf, self.struct.wq, self.N * self.K, torch.int8, (self.N, self.K))
+
+    @property
+    def col_absmax(self) -> torch.Tensor:   # N float32
+        return _view(self.buf, self.struct.col_absmax, self.N, torch.float32)
+
+    @property
+    def w_keep(self) -> torch.Tensor:       # n_keep x N fp16
+        return _view(self.buf, self.struct.w_keep, self.n_keep * self.N, torch.float16, (self.n_keep, self.N))
+
+    @property
+    def keep_idx(self) -> torch.Tensor:
+        return _view(self.buf, self.struct.keep_idx, self.n_keep, torch.int32)
+
+
+def prepare_weight(W: torch.Tensor, keep_idx=(), stream=None) -> PreparedWeight:
+    """Convert a K x N fp16 CUDA weight to int8 once ("converted to Int8" at load)."""
+    lib = _abi.load()
+    if not (W.is_cuda and W.dtype == torch.float16 and W.dim() == 2 and W.is_contiguous()):
+        raise ValueError("W must be a contiguous 2-D float16 CUDA tensor (K x N)")
+    K, N = W.shape
+    keep = np.unique(np.asarray(keep_idx, dtype=np.int64).ravel()).astype(np.int32)
+    nbytes = lib.int8mm_weight_bytes(K, N, int(keep.size))
+    if nbytes == 0:
+        raise Int8mmError(1, f"int8mm_weight_bytes(K={K}, N={N}, n_keep={keep.size})")
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    st = _abi.Weight()
+    kp = keep.ctypes.data_as(ctypes.c_void_p) if keep.size else None
+    with torch.cuda.device(W.device):
+        _abi.check(lib.int8mm_prepare_weight(ctypes.c_void_p(W.data_ptr()), K, N, kp, int(keep.size),
+                                             ctypes.c_void_p(buf.data_ptr()), nbytes, ctypes.byref(st),
+                                             _stream(stream)), "int8mm_prepare_weight")
+    return PreparedWeight(buf, st)
+
+
+class Workspace:
+    """Device scratch of one forward shape; zero-filled at creation."""
+
+    def __init__(self, M: int, K: int, N: int, max_outliers: int | None = None, device=None):
+        lib = _abi.load()
+        self.M, self.K, self.N = M, K, N
+        self.max_outliers = K if max_outliers is None else int(max_outliers)
+        self.nbytes = lib.int8mm_workspace_bytes(M, K, N, self.max_outliers)
+        if self.nbytes == 0:
+            raise Int8mmError(1, f"int8mm_workspace_bytes(M={M}, K={K}, N={N}, max_outliers={self.max_outliers})")
+        self.buf = torch.zeros(self.nbytes, dtype=torch.uint8, device=device or "cuda")
+
+    def reset(self, stream=None) -> None:
+        """Zero the workspace again (needed after a forward reported a device error)."""
+        with torch.cuda.device(self.buf.device):
+            _abi.check(_abi.load().int8mm_workspace_init(ctypes.c_void_p(self.buf.data_ptr()), self.nbytes,
+                                                         _stream(stream)), "int8mm_workspace_init")
+
+    def view(self) -> dict:
+        """Torch views of the intermediates the last forward left in the workspace."""
+        v = _abi.WorkspaceView()
+        _abi.check(_abi.load().int8mm_workspace_view_get(ctypes.c_void_p(self.buf.data_ptr()), self.nbytes, self.M,
+                                                         self.K, self.N, self.max_outliers, ctypes.byref(v)),
+                   "int8mm_workspace_view_get")
+        b = self.buf
+        return {
+            "status": _view(b, v.status, 1, torch.int32),
+            "n_outliers": _view(b, v.n_outliers, 1, torch.int32),
+            "outlier_idx": _view(b, v.outlier_idx, self.K, torch.int32),
+            "row_absmax": _view(b, v.row_absmax, self.M, torch.float32),
+            "xq": _view(b, v.xq, self.M * self.K, torch.int8, (self.M, self.K)),
+            "xo": _view(b, v.xo, self.M * v.kp, torch.float16, (self.M, v.kp)) if v.kp else None,
+            "kp": v.kp,
+        }
+
+
+def forward(X: torch.Tensor, w: PreparedWeight, threshold: float = 6.0, *, max_outliers: int | None = None,
+            out: torch.Tensor | None = None, workspace: Workspace | None = None, path: str = "auto",
+            acc_out: torch.Tensor | None = None, wait_limit_ns: int = 0, test_flags: int = 0,
+            stream=None) -> torch.Tensor:
+    """Y = X W by LLM.int8().  X: M x K fp16.  A CPU X is copied to the GPU and
+    the result copied back (end to end); a CUDA X stays on its device."""
+    lib = _abi.load()
+    on_host = not X.is_cuda
+    dev = w.buf.device
+    if X.dtype != torch.float16 or X.dim() != 2 or X.shape[1] != w.K:
+        raise ValueError(f"X must be float16 of shape (M, {w.K})")
+    Xd = X.to(dev, non_blocking=True) if on_host else X
+    if not Xd.is_contiguous():
+        raise ValueError("X must be contiguous")
+    M = Xd.shape[0]
+    if workspace is None:
+        workspace = Workspace(M, w.K, w.N, max_outliers, device=dev)
+    if (workspace.M, workspace.K, workspace.N) != (M, w.K, w.N):
+        raise ValueError("workspace was made for another shape")
+    Y = out if (out is not None and not on_host) else torch.empty(M, w.N, dtype=torch.float16, device=dev)
+    opts = _abi.ForwardOpts(_PATHS[path], ctypes.c_void_p(acc_out.data_ptr()) if acc_out is not None else None,
+                            int(wait_limit_ns), None, None, int(test_flags))
+    with torch.cuda.device(dev):
+        _abi.check(lib.int8mm_forward_ex(ctypes.c_void_p(Xd.data_ptr()), M, ctypes.byref(w.struct), float(threshold),
+                                         workspace.max_outliers, ctypes.c_void_p(Y.data_ptr()),
+                                         ctypes.c_void_p(workspace.buf.data_ptr()), workspace.nbytes,
+                                         ctypes.byref(opts), _stream(stream)), "int8mm_forward")
+    if on_host:
+        host = out if out is not None else torch.empty(M, w.N, dtype=torch.float16, pin_memory=True)
+        host.copy_(Y, non_blocking=True)
+        (stream or torch.cuda.current_stream()).synchronize()
+        return host
+    return Y
+
+
+def device_status(workspace: Workspace, stream=None) -> tuple[int, int]:
+    """(status code, detected outlier count) of the last forward; syncs the stream."""
+    n = ctypes.c_int32(0)
+    with torch.cuda.device(workspace.buf.device):
+        st = _abi.load().int8mm_get_device_status(ctypes.c_void_p(workspace.buf.data_ptr()), _stream(stream),
+                                                  ctypes.byref(n))
+    return int(st), int(n.value)

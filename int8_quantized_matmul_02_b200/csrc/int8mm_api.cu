@@ -1,0 +1,526 @@
+// C-ABI of libint8mm: argument checks, buffer layouts, TMA descriptors and
+// kernel launches for the LLM.int8() matmul ("LLM.int8(): 8-bit Matrix
+// Multiplication for Transformers at Scale", abstract).  The declarations and
+// their contracts are in include/int8mm.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "int8mm.h"
+#include "decode_sm100.cuh"
+#include "gemm_sm100.cuh"
+#include "quant_kernels.cuh"
+
+namespace {
+
+using namespace i8mm;
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr uint64_t kDefaultWaitNs = 2000ull * 1000 * 1000;
+constexpr int kMaxK = 131072;
+constexpr int kMaxSmemOptin = 232448;  // 227 KB per block on sm_100
+constexpr int kMaxDecodeRows = 16;
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// ------------------------------------------------------------------ device facts
+
+struct DeviceInfo {
+    int sm_count = 0;
+    bool ok = false;
+    bool attrs_set = false;
+};
+std::mutex g_dev_mu;
+DeviceInfo g_dev[64];
+
+int8mm_status current_device(int* dev_out, DeviceInfo** info_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return INT8MM_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= 64) return INT8MM_ERR_UNSUPPORTED_DEVICE;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ok) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return INT8MM_ERR_CUDA;
+        }
+        if (major != 10 || minor != 0) return INT8MM_ERR_UNSUPPORTED_DEVICE;
+        d.sm_count = sms;
+        d.ok = true;
+    }
+    if (!d.attrs_set) {
+        if (cudaFuncSetAttribute(k_gemm_int8_sm100<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGemmSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(k_gemm_int8_sm100<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGemmSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(k_decode_int8_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kMaxSmemOptin) != cudaSuccess) {
+            cudaGetLastError();
+            return INT8MM_ERR_CUDA;
+        }
+        d.attrs_set = true;
+    }
+    *dev_out = dev;
+    *info_out = &d;
+    return INT8MM_OK;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// Row-major 2-D tensor of `outer` rows x `inner` elements with a 128-byte
+// swizzled box of box_outer rows x box_inner elements (box_inner * elem = 128).
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ layouts
+
+struct WeightLayout {
+    size_t wq, ca, w_keep, keep_idx, keep_slot, total;
+};
+
+WeightLayout weight_layout(int K, int N, int n_keep) {
+    WeightLayout L{};
+    size_t o = 0;
+    L.wq = o;
+    o = align_up(o + (size_t)N * K, 256);
+    L.ca = o;
+    o = align_up(o + (size_t)N * 4, 256);
+    L.w_keep = o;
+    o = align_up(o + (size_t)n_keep * N * 2, 256);
+    L.keep_idx = o;
+    o = align_up(o + (size_t)n_keep * 4, 256);
+    L.keep_slot = o;
+    o = align_up(o + (size_t)K * 4, 256);
+    L.total = o;
+    return L;
+}
+
+struct WsLayout {
+    size_t status, n_out, mask, idx, ra, xq, xo, wo, partial, counters, total;
+    int kp;
+};
+
+WsLayout ws_layout(int M, int K, int N, int max_outliers) {
+    WsLayout L{};
+    L.kp = (max_outliers + 63) / 64 * 64;
+    size_t o = 0;
+    L.status = 0;
+    L.n_out = 4;
+    o = 256;
+    L.mask = o;
+    o = align_up(o + (size_t)cdiv(K, 32) * 4, 256);
+    L.idx = o;
+    o = align_up(o + (size_t)K * 4, 256);
+    L.ra = o;
+    o = align_up(o + (size_t)M * 4, 256);
+    L.xq = o;
+    o = align_up(o + (size_t)M * K, 256);
+    L.xo = o;
+    o = align_up(o + (size_t)M * L.kp * 2, 256);
+    L.wo = o;
+    o = align_up(o + (size_t)N * L.kp * 2, 256);
+    L.partial = o;
+    L.counters = o;
+    if (M <= kMaxDecodeRows) {
+        o = align_up(o + (size_t)kMaxDecodeRows * N * 4, 256);
+        L.counters = o;
+        o = align_up(o + (size_t)cdiv(N, kDecTileN) * 4 * 4, 256);
+    }
+    L.total = o;
+    return L;
+}
+
+bool shape_ok(int M, int K, int N) {
+    return M >= 1 && K >= 16 && N >= 16 && K % 16 == 0 && N % 16 == 0 && K <= kMaxK;
+}
+
+template <typename Kern, typename... Args>
+cudaError_t launch(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+int8mm_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return INT8MM_OK;
+    cudaGetLastError();
+    return INT8MM_ERR_CUDA;
+}
+
+// Shared-memory plan of the decode kernel for (M, K, cap); false if it does not fit.
+struct DecodePlan {
+    int stages, groups;
+    uint32_t off_xq, off_mask, off_pre, off_list, off_bars, bytes;
+};
+
+bool decode_plan(int M, int K, int cap, DecodePlan* P) {
+    if (M > kMaxDecodeRows || K > 65536) return false;
+    const int groups = (M + 7) / 8;
+    const int kb = cdiv(K, 128);
+    const int nw = cdiv(K, 32);
+    const size_t xq = (size_t)(kb * groups + 1) * 1024;
+    const size_t mask = align_up((size_t)nw * 4, 16);
+    const size_t pre = align_up((size_t)nw * 4, 16);
+    const size_t list = align_up((size_t)std::min(K, std::max(cap, 1)) * 2, 16);
+    const size_t fixed = xq + mask + pre + list;
+    const int max_stages = 16;
+    for (int s = max_stages; s >= 3; --s) {
+        const size_t bars = (size_t)(2 * s + 6) * 8 + 128;
+        const size_t total = 1024 + (size_t)s * kDecStageBytes + fixed + bars;
+        if (total <= (size_t)kMaxSmemOptin) {
+            P->stages = s;
+            P->groups = groups;
+            size_t o = (size_t)s * kDecStageBytes;
+            P->off_xq = (uint32_t)o;
+            o += xq;
+            P->off_mask = (uint32_t)o;
+            o += mask;
+            P->off_pre = (uint32_t)o;
+            o += pre;
+            P->off_list = (uint32_t)o;
+            o += list;
+            P->off_bars = (uint32_t)align_up(o, 8);
+            P->bytes = (uint32_t)total;
+            return true;
+        }
+    }
+    return false;
+}
+
+}  // namespace
+
+// ====================================================================== C-ABI
+
+extern "C" {
+
+const char* int8mm_status_string(int8mm_status s) {
+    switch (s) {
+        case INT8MM_OK: return "INT8MM_OK";
+        case INT8MM_ERR_INVALID_ARGUMENT: return "INT8MM_ERR_INVALID_ARGUMENT";
+        case INT8MM_ERR_MISALIGNED: return "INT8MM_ERR_MISALIGNED";
+        case INT8MM_ERR_WORKSPACE_TOO_SMALL: return "INT8MM_ERR_WORKSPACE_TOO_SMALL";
+        case INT8MM_ERR_UNSUPPORTED_DEVICE: return "INT8MM_ERR_UNSUPPORTED_DEVICE";
+        case INT8MM_ERR_CUDA: return "INT8MM_ERR_CUDA";
+        case INT8MM_ERR_TIMEOUT: return "INT8MM_ERR_TIMEOUT";
+        case INT8MM_ERR_OUTLIER_OVERFLOW: return "INT8MM_ERR_OUTLIER_OVERFLOW";
+    }
+    return "INT8MM_UNKNOWN_STATUS";
+}
+
+int int8mm_version(void) { return kVersion; }
+
+size_t int8mm_weight_bytes(int K, int N, int n_keep) {
+    if (!shape_ok(1, K, N) || n_keep < 0 || n_keep > K) return 0;
+    return weight_layout(K, N, n_keep).total;
+}
+
+int8mm_status int8mm_prepare_weight(const uint16_t* W, int K, int N, const int32_t* keep_idx_host, int n_keep,
+                                    void* buf, size_t buf_bytes, int8mm_weight* out, void* stream) {
+    if (!W || !buf || !out || !shape_ok(1, K, N) || n_keep < 0 || n_keep > K || (n_keep > 0 && !keep_idx_host))
+        return INT8MM_ERR_INVALID_ARGUMENT;
+    for (int i = 0; i < n_keep; ++i) {
+        const int k = keep_idx_host[i];
+        if (k < 0 || k >= K || (i > 0 && k <= keep_idx_host[i - 1])) return INT8MM_ERR_INVALID_ARGUMENT;
+    }
+    if (!aligned(W, 16) || !aligned(buf, 256)) return INT8MM_ERR_MISALIGNED;
+    const WeightLayout L = weight_layout(K, N, n_keep);
+    if (buf_bytes < L.total) return INT8MM_ERR_WORKSPACE_TOO_SMALL;
+    int dev;
+    DeviceInfo* info;
+    int8mm_status st = current_device(&dev, &info);
+    if (st != INT8MM_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* b = static_cast<uint8_t*>(buf);
+
+    int8mm_weight w{};
+    w.K = K;
+    w.N = N;
+    w.n_keep = n_keep;
+    w.wq = reinterpret_cast<int8_t*>(b + L.wq);
+    w.col_absmax = reinterpret_cast<float*>(b + L.ca);
+    w.w_keep = reinterpret_cast<uint16_t*>(b + L.w_keep);
+    w.keep_idx = reinterpret_cast<int32_t*>(b + L.keep_idx);
+    w.keep_slot = reinterpret_cast<int32_t*>(b + L.keep_slot);
+
+    std::vector<int32_t> slot(K, -1);
+    for (int i = 0; i < n_keep; ++i) slot[keep_idx_host[i]] = i;
+
+    cudaError_t e = cudaMemsetAsync(w.col_absmax, 0, (size_t)N * 4, s);
+    if (e == cudaSuccess) {
+        const int ksplit = std::min(cdiv(K, 64), 128);
+        const int rows = cdiv(K, ksplit);
+        e = launch(k_col_absmax, dim3(cdiv(N, 2048), ksplit), dim3(256), 0, s, false, W, K, N, rows,
+                   reinterpret_cast<unsigned*>(w.col_absmax));
+    }
+    if (e == cudaSuccess)
+        e = launch(k_quant_weight, dim3(cdiv(N, 64), cdiv(K, 64)), dim3(256), 0, s, false, W, K, N,
+                   (const float*)w.col_absmax, w.wq);
+    if (e == cudaSuccess && n_keep > 0)
+        e = cudaMemcpyAsync(w.keep_idx, keep_idx_host, (size_t)n_keep * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(w.keep_slot, slot.data(), (size_t)K * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && n_keep > 0)
+        e = launch(k_copy_keep_rows, dim3(n_keep), dim3(256), 0, s, false, W, N, (const int32_t*)w.keep_idx,
+                   w.w_keep);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);  // the host arrays above go out of scope
+    if (e != cudaSuccess) return cuda_status(e);
+    *out = w;
+    return INT8MM_OK;
+}
+
+size_t int8mm_workspace_bytes(int M, int K, int N, int max_outliers) {
+    if (!shape_ok(M, K, N) || max_outliers < 0 || max_outliers > K) return 0;
+    return ws_layout(M, K, N, max_outliers).total;
+}
+
+int8mm_status int8mm_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+    if (!ws || ws_bytes == 0) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!aligned(ws, 256)) return INT8MM_ERR_MISALIGNED;
+    return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int8mm_status int8mm_workspace_view_get(void* ws, size_t ws_bytes, int M, int K, int N, int max_outliers,
+                                        int8mm_workspace_view* out) {
+    if (!ws || !out || !shape_ok(M, K, N) || max_outliers < 0 || max_outliers > K)
+        return INT8MM_ERR_INVALID_ARGUMENT;
+    const WsLayout L = ws_layout(M, K, N, max_outliers);
+    if (ws_bytes < L.total) return INT8MM_ERR_WORKSPACE_TOO_SMALL;
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    out->status = reinterpret_cast<int32_t*>(b + L.status);
+    out->n_outliers = reinterpret_cast<int32_t*>(b + L.n_out);
+    out->outlier_idx = reinterpret_cast<int32_t*>(b + L.idx);
+    out->row_absmax = reinterpret_cast<float*>(b + L.ra);
+    out->xq = reinterpret_cast<int8_t*>(b + L.xq);
+    out->xo = reinterpret_cast<uint16_t*>(b + L.xo);
+    out->kp = L.kp;
+    return INT8MM_OK;
+}
+
+int8mm_status int8mm_get_device_status(const void* ws, void* stream, int32_t* n_outliers) {
+    if (!ws) return INT8MM_ERR_INVALID_ARGUMENT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int32_t h[2] = {0, 0};
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = cudaMemcpy(h, ws, sizeof(h), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (n_outliers) *n_outliers = h[1];
+    if (h[0] & kStatusTimeout) return INT8MM_ERR_TIMEOUT;
+    if (h[0] & kStatusOverflow) return INT8MM_ERR_OUTLIER_OVERFLOW;
+    return INT8MM_OK;
+}
+
+int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w, float threshold,
+                                int max_outliers, uint16_t* Y, void* ws, size_t ws_bytes,
+                                const int8mm_forward_opts* opts, void* stream) {
+    if (!X || !w || !Y || !ws || !w->wq || !w->col_absmax || !w->keep_slot) return INT8MM_ERR_INVALID_ARGUMENT;
+    const int K = w->K, N = w->N;
+    if (!shape_ok(M, K, N) || max_outliers < 0 || max_outliers > K) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!(threshold > 0.0f)) return INT8MM_ERR_INVALID_ARGUMENT;  // also rejects NaN
+    const int path = opts ? opts->path : INT8MM_PATH_AUTO;
+    if (path < INT8MM_PATH_AUTO || path > INT8MM_PATH_DECODE) return INT8MM_ERR_INVALID_ARGUMENT;
+    int32_t* acc_out = opts ? opts->acc_out : nullptr;
+    cudaEvent_t ev0 = opts ? reinterpret_cast<cudaEvent_t>(opts->main_start_event) : nullptr;
+    cudaEvent_t ev1 = opts ? reinterpret_cast<cudaEvent_t>(opts->main_stop_event) : nullptr;
+    if ((ev0 == nullptr) != (ev1 == nullptr)) return INT8MM_ERR_INVALID_ARGUMENT;
+    const bool timed = ev0 != nullptr;
+    const uint32_t test_flags = opts ? opts->test_flags : 0u;
+    const uint64_t wait_ns = (opts && opts->wait_limit_ns) ? opts->wait_limit_ns : kDefaultWaitNs;
+    if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ws, 256) || !aligned(w->wq, 256) ||
+        (acc_out && !aligned(acc_out, 16)))
+        return INT8MM_ERR_MISALIGNED;
+    const WsLayout L = ws_layout(M, K, N, max_outliers);
+    if (ws_bytes < L.total) return INT8MM_ERR_WORKSPACE_TOO_SMALL;
+
+    DecodePlan dp{};
+    const bool decode_fits = decode_plan(M, K, max_outliers, &dp);
+    bool use_decode;
+    if (path == INT8MM_PATH_DECODE) {
+        if (!decode_fits) return INT8MM_ERR_INVALID_ARGUMENT;
+        use_decode = true;
+    } else if (path == INT8MM_PATH_GEMM) {
+        use_decode = false;
+    } else {
+        use_decode = decode_fits;
+    }
+
+    int dev;
+    DeviceInfo* info;
+    int8mm_status st = current_device(&dev, &info);
+    if (st != INT8MM_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    int* status = reinterpret_cast<int*>(b + L.status);
+    int32_t* n_out = reinterpret_cast<int32_t*>(b + L.n_out);
+    uint32_t* mask = reinterpret_cast<uint32_t*>(b + L.mask);
+    int32_t* idx = reinterpret_cast<int32_t*>(b + L.idx);
+    float* ra = reinterpret_cast<float*>(b + L.ra);
+    int8_t* xq = reinterpret_cast<int8_t*>(b + L.xq);
+    uint16_t* xo = reinterpret_cast<uint16_t*>(b + L.xo);
+    uint16_t* wo = reinterpret_cast<uint16_t*>(b + L.wo);
+
+    if (use_decode) {
+        CUtensorMap tm_w;
+        if (!make_map(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq, K, N, K, 128, kDecTileN))
+            return INT8MM_ERR_CUDA;
+        DecodeParams p{};
+        p.X = X;
+        p.M = M;
+        p.K = K;
+        p.N = N;
+        p.thr = threshold;
+        p.cap = max_outliers;
+        p.wq = w->wq;
+        p.ca = w->col_absmax;
+        p.w_keep = w->w_keep;
+        p.keep_slot = w->keep_slot;
+        p.Y = Y;
+        p.partial = reinterpret_cast<int32_t*>(b + L.partial);
+        p.counters = reinterpret_cast<int32_t*>(b + L.counters);
+        p.acc_out = acc_out;
+        p.idx_out = idx;
+        p.n_out = n_out;
+        p.ra_out = ra;
+        p.xq_out = xq;
+        p.status = status;
+        p.wait_limit_ns = wait_ns;
+        p.test_flags = test_flags;
+        p.num_tiles = cdiv(N, kDecTileN);
+        p.kb_per_tile = cdiv(K, 128);
+        p.stages = dp.stages;
+        p.groups = dp.groups;
+        p.off_xq = dp.off_xq;
+        p.off_mask = dp.off_mask;
+        p.off_pre = dp.off_pre;
+        p.off_list = dp.off_list;
+        p.off_bars = dp.off_bars;
+        const long long units = (long long)p.num_tiles * p.kb_per_tile;
+        const int grid = (int)std::min<long long>(units, info->sm_count);
+        cudaError_t e = timed ? cudaEventRecord(ev0, s) : cudaSuccess;
+        if (e == cudaSuccess)
+            e = launch(k_decode_int8_sm100, dim3(grid), dim3(kDecThreads), dp.bytes, s, !timed, tm_w, p);
+        if (e == cudaSuccess && timed) e = cudaEventRecord(ev1, s);
+        return cuda_status(e);
+    }
+
+    // ---- tiled path: detect -> quantise -> gather -> tcgen05 GEMM, PDL-chained
+    CUtensorMap tm_a, tm_b, tm_xo, tm_wo, tm_y;
+    const int kp = L.kp;
+    if (!make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, M, K, 128, kGemmBM) ||
+        !make_map(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq, K, N, K, 128, kGemmBN) ||
+        !make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Y, N, M, (uint64_t)N * 2, 64, 32))
+        return INT8MM_ERR_CUDA;
+    if (kp > 0) {
+        if (!make_map(&tm_xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xo, kp, M, (uint64_t)kp * 2, 64, kGemmBM) ||
+            !make_map(&tm_wo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wo, kp, N, (uint64_t)kp * 2, 64, kGemmBN))
+            return INT8MM_ERR_CUDA;
+    } else {
+        tm_xo = tm_a;  // never dereferenced: no outlier slices without capacity
+        tm_wo = tm_b;
+    }
+
+    const int sms = info->sm_count;
+    cudaError_t e;
+    {
+        const int gx = cdiv(K, 256);
+        int gy = std::max(1, std::min(cdiv(M, 8), cdiv(4 * sms, gx)));
+        int rows = cdiv(M, gy);
+        rows = (rows + 7) / 8 * 8;
+        gy = cdiv(M, rows);
+        e = launch(k_detect, dim3(gx, gy), dim3(256), 0, s, false, X, M, K, threshold, rows, mask);
+    }
+    if (e == cudaSuccess) {
+        const int grid = std::min(M, sms * 8);
+        const size_t smem = (size_t)cdiv(K, 32) * 8;
+        if (K <= 16384)
+            e = launch(k_quant_rows<true>, dim3(grid), dim3(256), smem, s, true, X, M, K, (const uint32_t*)mask,
+                       max_outliers, kp, xq, ra, xo, idx, n_out, status);
+        else
+            e = launch(k_quant_rows<false>, dim3(grid), dim3(256), smem, s, true, X, M, K, (const uint32_t*)mask,
+                       max_outliers, kp, xq, ra, xo, idx, n_out, status);
+    }
+    if (e == cudaSuccess)
+        e = launch(k_gather_wo, dim3(cdiv(N, 64)), dim3(256), 0, s, true, (const int8_t*)w->wq,
+                   (const float*)w->col_absmax, (const uint16_t*)w->w_keep, (const int32_t*)w->keep_slot, K, N,
+                   (const int32_t*)idx, (const int32_t*)n_out, max_outliers, kp, wo, mask);
+    if (e == cudaSuccess) {
+        GemmParams p{};
+        p.M = M;
+        p.N = N;
+        p.K = K;
+        p.num_m_blocks = cdiv(M, kGemmBM);
+        p.num_n_blocks = cdiv(N, kGemmBN);
+        p.num_tiles = p.num_m_blocks * p.num_n_blocks;
+        p.group_m = std::min(16, p.num_m_blocks);
+        p.kb_int8 = cdiv(K, 128);
+        p.n_outliers = n_out;
+        p.cap = max_outliers;
+        p.ra = ra;
+        p.ca = w->col_absmax;
+        p.acc_out = acc_out;
+        p.status = status;
+        p.wait_limit_ns = wait_ns;
+        p.test_flags = test_flags;
+        const int grid = std::min(p.num_tiles, sms);
+        if (timed) e = cudaEventRecord(ev0, s);
+        if (e == cudaSuccess)
+            e = acc_out ? launch(k_gemm_int8_sm100<true>, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, s,
+                                 !timed, tm_a, tm_b, tm_xo, tm_wo, tm_y, p)
+                        : launch(k_gemm_int8_sm100<false>, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, s,
+                                 !timed, tm_a, tm_b, tm_xo, tm_wo, tm_y, p);
+        if (e == cudaSuccess && timed) e = cudaEventRecord(ev1, s);
+    }
+    return cuda_status(e);
+}
+
+int8mm_status int8mm_forward(const uint16_t* X, int M, const int8mm_weight* w, float threshold, int max_outliers,
+                             uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
+    return int8mm_forward_ex(X, M, w, threshold, max_outliers, Y, ws, ws_bytes, nullptr, stream);
+}
+
+}  // extern "C"

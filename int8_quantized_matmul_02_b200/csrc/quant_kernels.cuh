@@ -1,0 +1,374 @@
+// Bandwidth-bound steps of the LLM.int8() forward pass and the one-time weight
+// conversion ("LLM.int8(): 8-bit Matrix Multiplication for Transformers at
+// Scale", abstract):
+//   k_col_absmax / k_quant_weight   -- per-output-channel absmax int8 weight (c)
+//   k_detect                        -- outlier feature columns of X (a)
+//   k_quant_rows                    -- row absmax int8 X without the outlier
+//                                      columns, plus the fp16 outlier columns (b)
+//   k_gather_wo                     -- fp16 weight rows of the outlier dims (d)
+// All loads of X / W are 16-byte vectors along the contiguous dimension.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "sm100_ptx.cuh"
+
+namespace i8mm {
+
+// |x| as a comparable integer: the fp16 sign bit cleared, NaN mapped to 0 so
+// that a NaN never wins a max and never counts as an outlier.
+__device__ __forceinline__ uint32_t abs_bits2(uint32_t two_halves) {
+    uint32_t a = two_halves & 0x7FFF7FFFu;
+    uint32_t not_nan = __vcmpleu2(a, 0x7C007C00u);  // 0xFFFF per lane where a <= +inf
+    return a & not_nan;
+}
+
+__device__ __forceinline__ float half_bits_to_float(uint32_t bits16) {
+    return __half2float(__ushort_as_half((unsigned short)bits16));
+}
+
+// round-half-even(x * scale) clamped to [-127, 127]; fp32 product as in the method.
+__device__ __forceinline__ int quant1(float x, float scale) {
+    int q = __float2int_rn(__fmul_rn(x, scale));
+    return max(-127, min(127, q));
+}
+
+// ------------------------------------------------------------------ weight
+
+// ca[n] = max_k |W[k, n]| as float bits via atomicMax (ca pre-zeroed).
+// Block: 256 threads, each 8 consecutive columns; grid (ceil(N/2048), ksplit).
+__global__ void k_col_absmax(const uint16_t* __restrict__ W, int K, int N, int rows_per_block,
+                             unsigned* __restrict__ ca_bits) {
+    const int col0 = (blockIdx.x * 256 + threadIdx.x) * 8;
+    if (col0 >= N) return;
+    const int k0 = blockIdx.y * rows_per_block;
+    const int k1 = min(K, k0 + rows_per_block);
+    uint32_t m[4] = {0, 0, 0, 0};
+    for (int k = k0; k < k1; ++k) {
+        uint4 v = __ldg(reinterpret_cast<const uint4*>(W + (size_t)k * N + col0));
+        m[0] = __vmaxu2(m[0], abs_bits2(v.x));
+        m[1] = __vmaxu2(m[1], abs_bits2(v.y));
+        m[2] = __vmaxu2(m[2], abs_bits2(v.z));
+        m[3] = __vmaxu2(m[3], abs_bits2(v.w));
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        atomicMax(&ca_bits[col0 + 2 * i], __float_as_uint(half_bits_to_float(m[i] & 0xFFFF)));
+        atomicMax(&ca_bits[col0 + 2 * i + 1], __float_as_uint(half_bits_to_float(m[i] >> 16)));
+    }
+}
+
+// Wq[n, k] = round_half_even(W[k, n] * (127 / ca[n])), transposed through a
+// 64 x 64 shared tile.  Block 256 threads, grid (ceil(N/64), ceil(K/64)).
+__global__ void k_quant_weight(const uint16_t* __restrict__ W, int K, int N, const float* __restrict__ ca,
+                               int8_t* __restrict__ Wq) {
+    __shared__ uint16_t tile[64][64 + 8];
+    const int n0 = blockIdx.x * 64, k0 = blockIdx.y * 64;
+    const int t = threadIdx.x;
+    // load 64 rows (k) x 64 cols (n): 512 chunks of 8 halves
+    for (int c = t; c < 512; c += 256) {
+        int r = c >> 3, cc = (c & 7) * 8;
+        int k = k0 + r, n = n0 + cc;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (k < K && n < N) v = __ldg(reinterpret_cast<const uint4*>(W + (size_t)k * N + n));
+        *reinterpret_cast<uint4*>(&tile[r][cc]) = v;
+    }
+    __syncthreads();
+    // write 64 rows (n) x 64 bytes (k): thread -> (n = t/4, 16 k's)
+    const int nl = t >> 2, kl = (t & 3) * 16;
+    const int n = n0 + nl;
+    if (n >= N) return;
+    const float a = ca[n];
+    const float scale = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+    uint32_t packed[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            int q = a > 0.0f ? quant1(half_bits_to_float(tile[kl + 4 * w + b][nl]), scale) : 0;
+            word |= ((uint32_t)(q & 0xFF)) << (8 * b);
+        }
+        packed[w] = word;
+    }
+    const int k = k0 + kl;
+    if (k < K)  // K % 16 == 0, so the 16-byte group is entirely in or out
+        *reinterpret_cast<uint4*>(Wq + (size_t)n * K + k) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+}
+
+// w_keep[i, :] = W[keep_idx[i], :]; one block per kept row.
+__global__ void k_copy_keep_rows(const uint16_t* __restrict__ W, int N, const int32_t* __restrict__ keep_idx,
+                                 uint16_t* __restrict__ w_keep) {
+    const int i = blockIdx.x;
+    const uint4* src = reinterpret_cast<const uint4*>(W + (size_t)keep_idx[i] * N);
+    uint4* dst = reinterpret_cast<uint4*>(w_keep + (size_t)i * N);
+    for (int c = threadIdx.x; c < N / 8; c += blockDim.x) dst[c] = __ldg(src + c);
+}
+
+// ------------------------------------------------------------------ (a) detect
+
+// One pass over X: column k is an outlier when max_m |X[m, k]| >= thr.
+// Block 256 threads = 8 warps over 256 columns (8 per lane); warps stride over
+// rows [row0, row1).  Flags are OR-ed into the bitmask (bit k of word k/32).
+__global__ void __launch_bounds__(256) k_detect(const uint16_t* __restrict__ X, int M, int K, float thr,
+                                                int rows_per_block, uint32_t* __restrict__ mask) {
+    pdl_launch_dependents();
+    __shared__ uint32_t red[8][32][4];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int col0 = blockIdx.x * 256 + lane * 8;
+    const int row0 = blockIdx.y * rows_per_block;
+    const int row1 = min(M, row0 + rows_per_block);
+    uint32_t m[4] = {0, 0, 0, 0};
+    if (col0 < K) {
+        for (int r = row0 + warp; r < row1; r += 8) {
+            uint4 v = __ldg(reinterpret_cast<const uint4*>(X + (size_t)r * K + col0));
+            m[0] = __vmaxu2(m[0], abs_bits2(v.x));
+            m[1] = __vmaxu2(m[1], abs_bits2(v.y));
+            m[2] = __vmaxu2(m[2], abs_bits2(v.z));
+            m[3] = __vmaxu2(m[3], abs_bits2(v.w));
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) red[warp][lane][i] = m[i];
+    __syncthreads();
+    if (warp != 0) return;
+#pragma unroll
+    for (int w = 1; w < 8; ++w)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m[i] = __vmaxu2(m[i], red[w][lane][i]);
+    uint32_t flags = 0;  // 8 bits, one per column of this lane
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (half_bits_to_float(m[i] & 0xFFFF) >= thr) flags |= 1u << (2 * i);
+        if (half_bits_to_float(m[i] >> 16) >= thr) flags |= 1u << (2 * i + 1);
+    }
+    if (col0 >= K) flags = 0;
+    // word j of this block = lanes 4j..4j+3
+    uint32_t f1 = __shfl_down_sync(0xffffffffu, flags, 1);
+    uint32_t f2 = __shfl_down_sync(0xffffffffu, flags, 2);
+    uint32_t f3 = __shfl_down_sync(0xffffffffu, flags, 3);
+    if ((lane & 3) == 0) {
+        uint32_t word = flags | (f1 << 8) | (f2 << 16) | (f3 << 24);
+        int wi = (blockIdx.x * 256 + lane * 8) >> 5;
+        if (word && wi * 32 < K) atomicOr(&mask[wi], word);
+    }
+}
+
+// ------------------------------------------------------------------ (b) quantise rows
+
+// Max |x| over the non-outlier columns of one 8-column chunk c (as fp16 bits).
+__device__ __forceinline__ uint32_t chunk_inlier_absmax(uint4 v, const uint32_t* smask, int c) {
+    const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;  // outlier flags of columns 8c..8c+7
+    const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+    uint32_t amax = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t a = abs_bits2(h[j]);
+        const uint32_t lo = ((fl >> (2 * j)) & 1u) ? 0u : (a & 0xFFFFu);
+        const uint32_t hi = ((fl >> (2 * j + 1)) & 1u) ? 0u : (a >> 16);
+        amax = max(amax, max(lo, hi));
+    }
+    return amax;
+}
+
+// Quantise one 8-column chunk c of a row; outlier columns give 0 and are
+// copied to their slot of the row's fp16 outlier vector.
+__device__ __forceinline__ uint2 quant_chunk(uint4 v, const uint32_t* smask, const int* spre, int c, float rmax,
+                                            float scale, int n_eff, uint16_t* xo_row) {
+    const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
+    const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t bits = (h[j >> 1] >> ((j & 1) * 16)) & 0xFFFFu;
+        int q = 0;
+        if (!((fl >> j) & 1u)) {
+            if (rmax > 0.0f) q = quant1(half_bits_to_float(bits), scale);
+        } else {
+            const int k = c * 8 + j;
+            const int w = k >> 5;
+            const int slot = spre[w] + __popc(smask[w] & ((1u << (k & 31)) - 1u));
+            if (slot < n_eff) xo_row[slot] = (uint16_t)bits;
+        }
+        out[j >> 2] |= ((uint32_t)(q & 0xFF)) << ((j & 3) * 8);
+    }
+    return make_uint2(out[0], out[1]);
+}
+
+// Per row m: ra[m] = max over non-outlier columns of |X[m,k]|,
+// Xq[m,k] = outlier ? 0 : q(X[m,k]), Xo[m, slot(k)] = X[m,k] for outlier k,
+// with Xo zero-padded to a multiple of 64 columns.  Block 0 also writes the
+// ascending outlier list, the count and the overflow flag.
+// Block: 256 threads; the grid strides over rows.  kRegs: the row fits in 8
+// 16-byte chunks per thread (K <= 16384) and is read once.
+template <bool kRegs>
+__global__ void __launch_bounds__(256, 2) k_quant_rows(const uint16_t* __restrict__ X, int M, int K,
+                                                    const uint32_t* __restrict__ mask, int cap, int kp,
+                                                    int8_t* __restrict__ Xq, float* __restrict__ ra,
+                                                    uint16_t* __restrict__ Xo, int32_t* __restrict__ idx,
+                                                    int32_t* __restrict__ n_out, int* __restrict__ status) {
+    extern __shared__ uint32_t qsm[];
+    const int nw = (K + 31) / 32;
+    uint32_t* smask = qsm;          // nw words
+    int* spre = reinterpret_cast<int*>(qsm + nw);  // nw exclusive prefix counts
+    __shared__ uint32_t red[8];
+    __shared__ int total_sh;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    pdl_wait();  // the outlier bitmask comes from k_detect
+    pdl_launch_dependents();
+
+    // exclusive scan of popcounts over the mask words
+    int carry = 0;
+    for (int base = 0; base < nw; base += 256) {
+        int w = base + tid;
+        uint32_t word = w < nw ? mask[w] : 0u;
+        if (w < nw) smask[w] = word;
+        int c = __popc(word);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) red[warp] = incl;
+        __syncthreads();
+        int wsum = 0;
+        for (int i = 0; i < warp; ++i) wsum += red[i];
+        int blk_total = 0;
+        for (int i = 0; i < 8; ++i) blk_total += red[i];
+        if (w < nw) spre[w] = carry + wsum + incl - c;
+        carry += blk_total;
+        __syncthreads();
+    }
+    if (tid == 0) total_sh = carry;
+    __syncthreads();
+    const int total = total_sh;
+    const int n_eff = min(total, cap);
+    const int n_pad = min(kp, (n_eff + 63) / 64 * 64);
+
+    if (blockIdx.x == 0) {
+        if (tid == 0) {
+            *n_out = total;
+            if (total > cap) atomicOr(status, kStatusOverflow);
+        }
+        for (int w = tid; w < nw; w += 256) {
+            uint32_t word = smask[w];
+            int s = spre[w];
+            while (word) {
+                int b = __ffs(word) - 1;
+                idx[s++] = w * 32 + b;
+                word &= word - 1;
+            }
+        }
+    }
+
+    const int nchunk = K / 8;
+    for (int m = blockIdx.x; m < M; m += gridDim.x) {
+        const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)m * K);
+        uint4 regs[kRegs ? 8 : 1];
+        uint32_t amax = 0;
+        if constexpr (kRegs) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int c = tid + i * 256;
+                if (c < nchunk) {
+                    regs[i] = __ldg(xr + c);
+                    amax = max(amax, chunk_inlier_absmax(regs[i], smask, c));
+                }
+            }
+        } else {
+            for (int c = tid; c < nchunk; c += 256) amax = max(amax, chunk_inlier_absmax(__ldg(xr + c), smask, c));
+        }
+        // block max
+        amax = __reduce_max_sync(0xffffffffu, amax);
+        __syncthreads();
+        if (lane == 0) red[warp] = amax;
+        __syncthreads();
+        uint32_t bm = red[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) bm = max(bm, red[i]);
+        const float rmax = half_bits_to_float(bm);
+        const float scale = rmax > 0.0f ? __fdiv_rn(127.0f, rmax) : 0.0f;
+        if (tid == 0) ra[m] = rmax;
+        uint2* qr = reinterpret_cast<uint2*>(Xq + (size_t)m * K);
+        uint16_t* xo_row = Xo + (size_t)m * kp;
+        if constexpr (kRegs) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int c = tid + i * 256;
+                if (c < nchunk) qr[c] = quant_chunk(regs[i], smask, spre, c, rmax, scale, n_eff, xo_row);
+            }
+        } else {
+            for (int c = tid; c < nchunk; c += 256)
+                qr[c] = quant_chunk(__ldg(xr + c), smask, spre, c, rmax, scale, n_eff, xo_row);
+        }
+        for (int j = n_eff + tid; j < n_pad; j += 256) xo_row[j] = 0;
+    }
+}
+
+// ------------------------------------------------------------------ (d) outlier weight rows
+
+// Wo[n, j] (N x kp fp16, K-major) = the fp16 weight row of outlier j: the kept
+// row W[idx[j], n] when idx[j] was kept at preparation, else the dequantised
+// value fp16(Wq[n, idx[j]] * ca[n] / 127); zero for n_eff <= j < pad64(n_eff).
+// Block 256 threads over 64 output channels; block 0 clears the outlier
+// bitmask for the next call.
+__global__ void __launch_bounds__(256) k_gather_wo(const int8_t* __restrict__ Wq, const float* __restrict__ ca,
+                                                   const uint16_t* __restrict__ w_keep,
+                                                   const int32_t* __restrict__ keep_slot, int K, int N,
+                                                   const int32_t* __restrict__ idx,
+                                                   const int32_t* __restrict__ n_out, int cap, int kp,
+                                                   uint16_t* __restrict__ Wo, uint32_t* __restrict__ mask) {
+    __shared__ uint16_t tile[64][64 + 8];
+    __shared__ int sidx[64];
+    __shared__ int sslot[64];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int tid = threadIdx.x;
+    if (blockIdx.x == 0)
+        for (int w = tid; w < (K + 31) / 32; w += 256) mask[w] = 0u;
+    const int n_eff = min(*n_out, cap);
+    const int n_pad = min(kp, (n_eff + 63) / 64 * 64);
+    const int n0 = blockIdx.x * 64;
+    for (int j0 = 0; j0 < n_pad; j0 += 64) {
+        __syncthreads();
+        if (tid < 64) {
+            int j = j0 + tid;
+            int k = j < n_eff ? idx[j] : -1;
+            sidx[tid] = k;
+            sslot[tid] = k >= 0 ? keep_slot[k] : -1;
+        }
+        __syncthreads();
+        // fill tile[j][n]: coalesced along n
+        for (int e = tid; e < 64 * 64; e += 256) {
+            int jl = e >> 6, nl = e & 63;
+            int n = n0 + nl, k = sidx[jl], slot = sslot[jl];
+            uint16_t v = 0;
+            if (k >= 0 && n < N) {
+                if (slot >= 0) {
+                    v = w_keep[(size_t)slot * N + n];
+                } else {
+                    float t = __fmul_rn((float)Wq[(size_t)n * K + k], ca[n]);
+                    v = __half_as_ushort(__float2half_rn(__fdiv_rn(t, 127.0f)));
+                }
+            }
+            tile[jl][nl] = v;
+        }
+        __syncthreads();
+        // write Wo[n][j0 .. j0+64): 64 rows x 128 bytes, 8 threads per row
+        for (int e = tid; e < 64 * 8; e += 256) {
+            int nl = e >> 3, c = (e & 7) * 8;
+            int n = n0 + nl;
+            if (n >= N) continue;
+            uint32_t w4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                w4[i] = (uint32_t)tile[c + 2 * i][nl] | ((uint32_t)tile[c + 2 * i + 1][nl] << 16);
+            *reinterpret_cast<uint4*>(Wo + (size_t)n * kp + j0 + c) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+    }
+}
+
+}  // namespace i8mm

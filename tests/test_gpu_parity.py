@@ -1,0 +1,206 @@
+"""GPU parity: the CUDA path through the C-ABI against the CPU oracle on the
+same seeded inputs (outlier list, int8 codes, scales and int32 sums
+bit-exact; fp16 Y within 2^-9 |y| + 1e-3 rms)."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import int8_quantized_matmul_02_b200 as i8
+from int8_quantized_matmul_02_b200 import synth
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu(cuda_ok):
+    torch.manual_seed(0)
+    yield
+
+
+def _run_case(M, K, N, n_seed, thr=6.0, path="auto", keep="seeded", cap=None, seed=0, mode="element",
+              lo=10.0, hi=60.0):
+    X, W, cols = synth.make_case(M, K, N, n_seed=n_seed, lo=lo, hi=hi, mode=mode, seed=seed)
+    keep_idx = {"seeded": cols, "none": [], "all": list(range(K))}[keep]
+    w = parity.gpu_prepare(W, keep_idx)
+    prep, r = parity.oracle_full(X, W, keep_idx, thr)
+    parity.check_weight(w, prep)
+    g = parity.gpu_forward(X, w, thr, path=path, cap=cap)
+    return parity.check_forward_full(g, r), r
+
+
+# ------------------------------------------------------------------ tiled GEMM path
+
+@pytest.mark.parametrize("M,K,N,n_seed", [
+    (16, 256, 384, 2),        # the tiny configuration's shape
+    (300, 1040, 784, 4),      # several 128 x 256 tiles, ragged M, N and K
+    (129, 512, 528, 3),
+    (256, 2048, 512, 7),
+])
+def test_gemm_path_matches_oracle(M, K, N, n_seed):
+    _run_case(M, K, N, n_seed, path="gemm")
+
+
+@pytest.mark.parametrize("M", [1, 8, 17, 64, 65, 129])
+def test_gemm_path_row_counts(M):
+    _run_case(M, 512, 272, 3, path="gemm", seed=M)
+
+
+@pytest.mark.parametrize("n_seed", [0, 1, 15, 16, 17, 64, 65])
+def test_gemm_path_outlier_counts(n_seed):
+    _, r = _run_case(160, 1024, 512, n_seed, path="gemm", seed=100 + n_seed)
+    assert r["idx"].size >= n_seed
+
+
+@pytest.mark.parametrize("keep", ["none", "all"])
+def test_gemm_path_kept_and_dequantised_rows(keep):
+    _run_case(130, 768, 528, 5, path="gemm", keep=keep, seed=7)
+
+
+def test_gemm_path_threshold_inf():
+    _, r = _run_case(200, 1024, 512, 6, thr=math.inf, path="gemm", seed=3)
+    assert r["idx"].size == 0
+
+
+def test_gemm_path_all_outliers():
+    # threshold below every |x|: every column is an outlier, the int8 part is empty
+    _, r = _run_case(96, 256, 272, 0, thr=1e-30, path="gemm", keep="all", seed=5)
+    assert r["idx"].size == 256
+
+
+def test_gemm_path_zero_rows_and_columns():
+    X, W, cols = synth.make_case(140, 512, 528, n_seed=3, seed=9)
+    X[5, :] = 0
+    X[:, 17] = 0
+    W[:, 33] = 0
+    w = parity.gpu_prepare(W, cols)
+    prep, r = parity.oracle_full(X, W, cols, 6.0)
+    parity.check_weight(w, prep)
+    parity.check_forward_full(parity.gpu_forward(X, w, 6.0, path="gemm"), r)
+
+
+# ------------------------------------------------------------------ fused decode path
+
+@pytest.mark.parametrize("M,K,N,n_seed", [
+    (1, 256, 384, 2),
+    (8, 4096, 1024, 6),
+    (9, 1024, 528, 3),
+    (16, 4112, 400, 5),       # K not a multiple of 128, N not a multiple of 128
+    (3, 2048, 11008, 1),
+])
+def test_decode_path_matches_oracle(M, K, N, n_seed):
+    _run_case(M, K, N, n_seed, path="decode", seed=M * 31 + K)
+
+
+@pytest.mark.parametrize("keep", ["none", "all"])
+def test_decode_path_kept_and_dequantised_rows(keep):
+    _run_case(8, 1024, 528, 4, path="decode", keep=keep, seed=11)
+
+
+def test_decode_path_threshold_inf_and_all_outliers():
+    _run_case(8, 1024, 272, 4, thr=math.inf, path="decode", seed=12)
+    _run_case(4, 256, 272, 0, thr=1e-30, path="decode", keep="all", seed=13)
+
+
+def test_decode_workspace_is_reusable():
+    """Split-K partial sums and tile counters return to zero after each call."""
+    M, K, N = 8, 4096, 2048
+    _, W, cols = synth.make_case(M, K, N, n_seed=4, seed=21)
+    w = parity.gpu_prepare(W, cols)
+    prep = oracle.prepare_weight(W.numpy(), cols)
+    ws = i8.Workspace(M, K, N)
+    for s in range(3):
+        X, _, _ = synth.make_case(M, K, N, n_seed=4, seed=21)  # same columns, new draws below
+        X = (X.float() * (1.0 + 0.1 * s)).half()
+        r = oracle.forward(X.numpy(), prep, 6.0)
+        parity.check_forward_full(parity.gpu_forward(X, w, 6.0, path="decode", ws=ws), r)
+
+
+def test_gemm_workspace_is_reusable():
+    M, K, N = 200, 1024, 528
+    X, W, cols = synth.make_case(M, K, N, n_seed=4, seed=22)
+    w = parity.gpu_prepare(W, cols)
+    prep = oracle.prepare_weight(W.numpy(), cols)
+    ws = i8.Workspace(M, K, N)
+    for s in range(3):
+        Xs = X.clone()
+        Xs[:, (s * 37) % K] = 30.0  # a different extra outlier column each call
+        r = oracle.forward(Xs.numpy(), prep, 6.0)
+        parity.check_forward_full(parity.gpu_forward(Xs, w, 6.0, path="gemm", ws=ws), r)
+
+
+def test_paths_agree():
+    X, W, cols = synth.make_case(12, 2048, 1040, n_seed=5, seed=23)
+    w = parity.gpu_prepare(W, cols)
+    a = parity.gpu_forward(X, w, 6.0, path="decode")
+    b = parity.gpu_forward(X, w, 6.0, path="gemm")
+    assert torch.equal(a["acc_dev"], b["acc_dev"])
+    parity.assert_y_close(a["Y_dev"].float().cpu().numpy(), b["Y_dev"].float().cpu().numpy())
+
+
+# ------------------------------------------------------------------ device-side errors
+
+@pytest.mark.parametrize("path", ["gemm", "decode"])
+def test_outlier_overflow_is_reported(path):
+    X, W, cols = synth.make_case(8, 1024, 512, n_seed=6, seed=30)
+    w = parity.gpu_prepare(W, cols)
+    ws = i8.Workspace(8, 1024, 512, max_outliers=2)
+    i8.forward(X.cuda(), w, 6.0, workspace=ws, path=path)
+    st, n = i8.device_status(ws)
+    assert st == 7 and n >= 6
+
+
+@pytest.mark.parametrize("path", ["gemm", "decode"])
+def test_wait_limit_reports_timeout_and_recovers(path):
+    """The main kernel withholds one internal signal, so a wait runs out after
+    its 50 ms limit: the kernel records a timeout and returns, and the context
+    stays usable for the next call."""
+    from int8_quantized_matmul_02_b200 import _abi
+
+    M = 8 if path == "decode" else 200
+    X, W, cols = synth.make_case(M, 2048, 1024, n_seed=3, seed=31)
+    w = parity.gpu_prepare(W, cols)
+    ws = i8.Workspace(M, 2048, 1024)
+    i8.forward(X.cuda(), w, 6.0, workspace=ws, path=path, wait_limit_ns=50_000_000,
+               test_flags=_abi.TEST_WITHHOLD_SIGNAL)
+    st, _ = i8.device_status(ws)
+    assert st == 6
+    ws.reset()
+    prep, r = parity.oracle_full(X, W, cols, 6.0)
+    parity.check_forward_full(parity.gpu_forward(X, w, 6.0, path=path, ws=ws), r)
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+def _full_size(name, cap=1024, full_oracle=False):
+    wl = synth.WORKLOADS[name]
+    X, W, cols = synth.make_inputs(wl)
+    w = parity.gpu_prepare(W, cols)
+    prep = oracle.prepare_weight(W.numpy(), cols)
+    parity.check_weight(w, prep)
+    cap = min(cap, wl.K)
+    g = parity.gpu_forward(X, w, wl.threshold, path="auto", cap=cap)
+    if full_oracle:
+        r = oracle.forward(X.numpy(), prep, wl.threshold)
+        parity.check_forward_full(g, r)
+        return r["idx"].size
+    steps = oracle.forward_steps_abc(X.numpy(), prep, wl.threshold)
+    pm, pn = synth.sample_points(wl.M, wl.N, 4096, seed=wl.seed, tiles=((128, 256), (128, 256)))
+    parity.check_forward_sampled(g, steps, prep, pm, pn)
+    return steps["idx"].size
+
+
+def test_full_size_decode():
+    n_o = _full_size("decode", full_oracle=True)
+    assert n_o >= 6
+
+
+@pytest.mark.parametrize("name", ["prefill", "175b", "qkv_o123", "qkv_inf"])
+def test_full_size_sampled(name):
+    n_o = _full_size(name)
+    assert n_o >= synth.WORKLOADS[name].n_seed
