@@ -156,6 +156,17 @@ def recorded_traffic(kernel: str, workload: str, units_scale: float = 1.0):
 
 # ----------------------------------------------------------------------------- our arm
 
+def event_pairs(n: int, stream):
+    """n (start, stop) timing events, created on the device (torch creates an
+    event lazily at its first record; the library records raw handles)."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for a, b in evs:
+        a.record(stream)
+        b.record(stream)
+    stream.synchronize()
+    return evs
+
+
 def algorithmic_bytes_decode(wl, n_o: int) -> float:
     """Minimum HBM bytes of one decode forward: Wq + ca + X + Y + the fp16
     weight rows of the outlier dims."""
@@ -172,7 +183,7 @@ def run_gemm_workload(wl, steps: int, warmup: int, dev, rank: int, cap: int):
     ws = i8.Workspace(wl.M, wl.K, wl.N, cap, device=dev)
     Y = torch.empty(wl.M, wl.N, dtype=torch.float16, device=dev)
     stream = torch.cuda.current_stream(dev)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    evs = event_pairs(steps, stream)
 
     def step(ev=None):
         lib = i8.library()
@@ -191,10 +202,6 @@ def run_gemm_workload(wl, steps: int, warmup: int, dev, rank: int, cap: int):
     st, n_o = i8.device_status(ws)
     if st != 0:
         raise RuntimeError(f"device status {st} after warm-up")
-    # make sure the events exist on the device before timing
-    for a, b in evs:
-        a.record(stream)
-        b.record(stream)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     barrier()
@@ -275,7 +282,7 @@ def run_decode(steps: int, warmup: int, dev, cap: int, copies: int = 8):
     if st != 0:
         raise RuntimeError(f"decode device status {st}")
     # (1) kernel-only timing: events around the fused kernel of every step
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    evs = event_pairs(steps, stream)
     for i in range(steps):
         fwd(i, evs[i])
     torch.cuda.synchronize(dev)
@@ -320,20 +327,18 @@ def barrier():
         torch.distributed.barrier()
 
 
-def max_over_ranks(v: float, dev) -> float:
-    if _pg is None:
-        return v
-    t = torch.tensor([v], dtype=torch.float64, device=dev)
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
-
-
-def sum_over_ranks(v: float, dev) -> float:
-    if _pg is None:
-        return v
-    t = torch.tensor([v], dtype=torch.float64, device=dev)
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
-    return float(t.item())
+def combine_ranks(per_step_s: float, units_per_step: float, dev, distributed: bool):
+    """Replicas: every rank times its own steps; the job's step time is the
+    slowest rank's and the job's throughput is all ranks' units over it.
+    Returns (max step seconds, job units per second)."""
+    if not distributed:
+        return per_step_s, units_per_step / per_step_s
+    t = torch.tensor([per_step_s, units_per_step], dtype=torch.float64, device=dev)
+    mx = t[:1].clone()
+    torch.distributed.all_reduce(mx, op=torch.distributed.ReduceOp.MAX)
+    tot = t[1:].clone()
+    torch.distributed.all_reduce(tot, op=torch.distributed.ReduceOp.SUM)
+    return float(mx.item()), float(tot.item()) / float(mx.item())
 
 
 # ----------------------------------------------------------------------------- CPU oracle timing
@@ -424,6 +429,10 @@ def main():
         return 1
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    # all timed work runs on one non-default stream (CUDA graphs cannot be
+    # captured on the legacy default stream)
+    bench_stream = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(bench_stream)
     if world > 1:
         import datetime
 
@@ -466,8 +475,7 @@ def main():
                 "frac_of_nominal_int8": (wl.ops / kern_s / 1e12) / NOMINAL_INT8_TOPS}
         launches = 4
 
-    per_step_max = max_over_ranks(per_step_s, dev)
-    value = sum_over_ranks(value_local * per_step_s / per_step_max, dev)
+    per_step_max, value = combine_ranks(per_step_s, value_local * per_step_s, dev, _pg is not None)
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = recorded_traffic("k_gemm_int8_sm100" if not small else "k_decode_int8_sm100", args.workload)
     roof["kernel"] = "k_gemm_int8_sm100" if not small else "k_decode_int8_sm100"
@@ -489,8 +497,13 @@ def main():
         e2e_ms, bi, bo = run_e2e(wl, r, max(3, args.steps // 4), dev)
         line["e2e"] = {"value": wl.ops / (e2e_ms * 1e-3) / 1e12 * world, "unit": unit, "h2d_bytes_per_step": bi,
                        "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms}
+        d = None
         if not args.no_decode:
-            d = run_decode(args.decode_steps, args.warmup, dev, min(args.max_outliers, 4096))
+            try:
+                d = run_decode(args.decode_steps, args.warmup, dev, min(args.max_outliers, 4096))
+            except Exception as exc:  # keep the headline line; say what failed
+                line["decode"] = {"error": f"{type(exc).__name__}: {exc}"}
+        if d is not None:
             dw = d["wl"]
             line["decode"] = {
                 "workload": WORKLOAD_NAMES["decode"], "metric": "HBM GB/s", "unit": "GB/s",
