@@ -29,6 +29,7 @@ EXPORTS = (
     "int8mm_status_string", "int8mm_version", "int8mm_weight_bytes", "int8mm_prepare_weight",
     "int8mm_workspace_bytes", "int8mm_workspace_init", "int8mm_forward", "int8mm_forward_ex",
     "int8mm_workspace_view_get", "int8mm_get_device_status",
+    "int8mm_forward_decode_noalloc", "int8mm_noalloc_device_status",
 )
 
 
@@ -96,6 +97,10 @@ def load(path: str | None = None):
     lib.int8mm_workspace_view_get.restype = I
     lib.int8mm_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
     lib.int8mm_get_device_status.restype = I
+    lib.int8mm_forward_decode_noalloc.argtypes = [P, I, ctypes.POINTER(Weight), F, P, P]
+    lib.int8mm_forward_decode_noalloc.restype = I
+    lib.int8mm_noalloc_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
+    lib.int8mm_noalloc_device_status.restype = I
     if path is None:
         _lib = lib
     return lib

@@ -234,6 +234,58 @@ bool decode_plan(int M, int K, int cap, DecodePlan* P) {
     return false;
 }
 
+// ------------------------------------------------------------------ no-allocation decode forward
+
+// Scratch of int8mm_forward_decode_noalloc: one array per GPU that loads the
+// library, zero at load, shared by every call of that entry point.
+constexpr size_t kNoAllocBytes = INT8MM_NOALLOC_SCRATCH_BYTES;
+constexpr int kNoAllocMaxK = 16384;
+constexpr int kNoAllocMaxN = 65536;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocBytes];
+
+// Layout inside the array: [status, count | counters | partial sums] (the
+// part cleared before every call), then the outlier list, ra and Xq.
+struct NoAllocLayout {
+    size_t counters, partial, clear_bytes, idx, ra, xq, total;
+};
+
+NoAllocLayout noalloc_layout(int M, int K, int N) {
+    NoAllocLayout L{};
+    size_t o = 256;
+    L.counters = o;
+    o = align_up(o + (size_t)cdiv(N, kDecTileN) * 4 * 4, 256);
+    L.partial = o;
+    o = align_up(o + (size_t)M * N * 4, 256);
+    L.clear_bytes = o;
+    L.idx = o;
+    o = align_up(o + (size_t)K * 4, 256);
+    L.ra = o;
+    o = align_up(o + (size_t)kMaxDecodeRows * 4, 256);
+    L.xq = o;
+    o = align_up(o + (size_t)M * K, 256);
+    L.total = o;
+    return L;
+}
+
+// Device address of the array on the current device, looked up once per
+// device (with that device current) by cudaGetSymbolAddress.
+std::mutex g_noalloc_mu;
+uint8_t* g_noalloc_ptr[64] = {};
+
+int8mm_status noalloc_scratch(int dev, uint8_t** out) {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return INT8MM_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = static_cast<uint8_t*>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return INT8MM_OK;
+}
+
 }  // namespace
 
 // ====================================================================== C-ABI
@@ -521,6 +573,82 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
 int8mm_status int8mm_forward(const uint16_t* X, int M, const int8mm_weight* w, float threshold, int max_outliers,
                              uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
     return int8mm_forward_ex(X, M, w, threshold, max_outliers, Y, ws, ws_bytes, nullptr, stream);
+}
+
+int8mm_status int8mm_forward_decode_noalloc(const uint16_t* X, int M, const int8mm_weight* w, float threshold,
+                                            uint16_t* Y, void* stream) {
+    if (!X || !w || !Y || !w->wq || !w->col_absmax || !w->keep_slot) return INT8MM_ERR_INVALID_ARGUMENT;
+    const int K = w->K, N = w->N;
+    if (!shape_ok(M, K, N) || M > kMaxDecodeRows || K > kNoAllocMaxK || N > kNoAllocMaxN)
+        return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!(threshold > 0.0f)) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(w->wq, 256)) return INT8MM_ERR_MISALIGNED;
+    const int cap = K;
+    DecodePlan dp{};
+    if (!decode_plan(M, K, cap, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
+    const NoAllocLayout L = noalloc_layout(M, K, N);
+    if (L.total > kNoAllocBytes) return INT8MM_ERR_INVALID_ARGUMENT;
+
+    int dev;
+    DeviceInfo* info;
+    int8mm_status st = current_device(&dev, &info);
+    if (st != INT8MM_OK) return st;
+    uint8_t* b = nullptr;
+    st = noalloc_scratch(dev, &b);
+    if (st != INT8MM_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+    CUtensorMap tm_w;
+    if (!make_map(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq, K, N, K, 128, kDecTileN)) return INT8MM_ERR_CUDA;
+    DecodeParams p{};
+    p.X = X;
+    p.M = M;
+    p.K = K;
+    p.N = N;
+    p.thr = threshold;
+    p.cap = cap;
+    p.wq = w->wq;
+    p.ca = w->col_absmax;
+    p.w_keep = w->w_keep;
+    p.keep_slot = w->keep_slot;
+    p.Y = Y;
+    p.partial = reinterpret_cast<int32_t*>(b + L.partial);
+    p.counters = reinterpret_cast<int32_t*>(b + L.counters);
+    p.acc_out = nullptr;
+    p.idx_out = reinterpret_cast<int32_t*>(b + L.idx);
+    p.n_out = reinterpret_cast<int32_t*>(b + 4);
+    p.ra_out = reinterpret_cast<float*>(b + L.ra);
+    p.xq_out = reinterpret_cast<int8_t*>(b + L.xq);
+    p.status = reinterpret_cast<int*>(b);
+    p.wait_limit_ns = kDefaultWaitNs;
+    p.test_flags = 0;
+    p.num_tiles = cdiv(N, kDecTileN);
+    p.kb_per_tile = cdiv(K, 128);
+    p.stages = dp.stages;
+    p.groups = dp.groups;
+    p.off_xq = dp.off_xq;
+    p.off_mask = dp.off_mask;
+    p.off_pre = dp.off_pre;
+    p.off_list = dp.off_list;
+    p.off_bars = dp.off_bars;
+    const long long units = (long long)p.num_tiles * p.kb_per_tile;
+    const int grid = (int)std::min<long long>(units, info->sm_count);
+    // status word, count, tile counters and the partial sums start at zero
+    cudaError_t e = cudaMemsetAsync(b, 0, L.clear_bytes, s);
+    if (e == cudaSuccess)
+        e = launch(k_decode_int8_sm100, dim3(grid), dim3(kDecThreads), dp.bytes, s, false, tm_w, p);
+    return cuda_status(e);
+}
+
+int8mm_status int8mm_noalloc_device_status(void* stream, int32_t* n_outliers) {
+    int dev;
+    DeviceInfo* info;
+    int8mm_status st = current_device(&dev, &info);
+    if (st != INT8MM_OK) return st;
+    uint8_t* b = nullptr;
+    st = noalloc_scratch(dev, &b);
+    if (st != INT8MM_OK) return st;
+    return int8mm_get_device_status(b, stream, n_outliers);
 }
 
 }  // extern "C"
