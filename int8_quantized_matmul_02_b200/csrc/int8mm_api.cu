@@ -173,19 +173,38 @@ bool shape_ok(int M, int K, int N) {
     return M >= 1 && K >= 16 && N >= 16 && K % 16 == 0 && N % 16 == 0 && K <= kMaxK;
 }
 
+// Launch with optional programmatic dependent launch (PDL) and an optional
+// thread-block cluster size along x.
 template <typename Kern, typename... Args>
-cudaError_t launch(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl, Args... args) {
+cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl, int cluster,
+                      Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = pdl ? attr : nullptr;
-    cfg.numAttrs = pdl ? 1 : 0;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    if (pdl) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    if (cluster > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = (unsigned)cluster;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = n ? attr : nullptr;
+    cfg.numAttrs = n;
     return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+template <typename Kern, typename... Args>
+cudaError_t launch(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl, Args... args) {
+    return launch_ex(kern, grid, block, smem, st, pdl, 1, args...);
 }
 
 int8mm_status cuda_status(cudaError_t e) {
@@ -194,25 +213,68 @@ int8mm_status cuda_status(cudaError_t e) {
     return INT8MM_ERR_CUDA;
 }
 
+// Value of a non-negative fp16 bit pattern h <= 0x7C00 (+inf).
+float fp16_value(uint32_t h) {
+    if (h == 0x7C00u) return INFINITY;
+    const int e = (int)(h >> 10), m = (int)(h & 0x3FFu);
+    return e == 0 ? std::ldexp((float)m, -24) : std::ldexp((float)(1024 + m), e - 25);
+}
+
+// Bits of the smallest fp16 value >= thr (thr > 0), replicated in both 16-bit
+// lanes; 0x7C01 (above +inf, below any NaN after masking) when none reaches it.
+// Non-negative fp16 bit patterns are ordered like their values, so a binary
+// search over [0, 0x7C00] finds it.
+uint32_t fp16_threshold_bits2(float thr) {
+    if (!(fp16_value(0x7C00u) >= thr)) return 0x7C017C01u;
+    uint32_t lo = 0, hi = 0x7C00u;  // fp16_value(hi) >= thr
+    while (lo < hi) {
+        const uint32_t mid = (lo + hi) / 2;
+        if (fp16_value(mid) >= thr)
+            hi = mid;
+        else
+            lo = mid + 1;
+    }
+    return lo | (lo << 16);
+}
+
+// K split of the decode kernel: one CTA per 128-channel tile when the tiles
+// alone fill at least half of the SMs, else enough K ranges per tile to do so.
+int decode_splits(int N, int K, int sms) {
+    const int tiles = cdiv(N, kDecTileN), kbs = cdiv(K, 128);
+    const int target = std::max(1, sms / 2);
+    return std::max(1, std::min(kbs, cdiv(target, tiles)));
+}
+
 // Shared-memory plan of the decode kernel for (M, K, cap); false if it does not fit.
 struct DecodePlan {
     int stages, groups;
-    uint32_t off_xq, off_mask, off_pre, off_list, off_bars, bytes;
+    uint32_t off_xq, off_mask, off_pre, off_list, off_xo, off_oslot, off_bars, off_xstage, bytes;
+    int cluster;
 };
 
-bool decode_plan(int M, int K, int cap, DecodePlan* P) {
+// CTAs per cluster that share the decode kernel's X-side steps.
+constexpr int kDecCluster = 4;
+
+// Shared-memory plan of the decode kernel for (M, K, cap) with `cluster` CTAs
+// sharing the X-side steps (each stages its share of X); false if it does not fit.
+bool decode_plan(int M, int K, int cap, int cluster, DecodePlan* P) {
     if (M > kMaxDecodeRows || K > 65536) return false;
     const int groups = (M + 7) / 8;
     const int kb = cdiv(K, 128);
     const int nw = cdiv(K, 32);
+    const int nchunk = K / 8;
     const size_t xq = (size_t)(kb * groups + 1) * 1024;
     const size_t mask = align_up((size_t)nw * 4, 16);
     const size_t pre = align_up((size_t)nw * 4, 16);
     const size_t list = align_up((size_t)std::min(K, std::max(cap, 1)) * 2, 16);
-    const size_t fixed = xq + mask + pre + list;
-    const int max_stages = 16;
-    for (int s = max_stages; s >= 3; --s) {
-        const size_t bars = (size_t)(2 * s + 6) * 8 + 128;
+    const size_t xo = (size_t)kDecSmemOutliers * 16 * 2;
+    const size_t oslot = (size_t)kDecSmemOutliers * 4;
+    const int nq = cdiv(cdiv(nchunk, 4), cluster) * 4;
+    const size_t xstage = cluster > 1 ? align_up((size_t)M * nq * 16, 128) : 0;
+    const size_t fixed = xq + mask + pre + list + xo + oslot + xstage;
+    const int min_stages = cluster > 1 ? 6 : 3;
+    for (int s = 16; s >= min_stages; --s) {
+        const size_t bars = (size_t)(2 * s + 6) * 8 + 256;
         const size_t total = 1024 + (size_t)s * kDecStageBytes + fixed + bars;
         if (total <= (size_t)kMaxSmemOptin) {
             P->stages = s;
@@ -220,16 +282,40 @@ bool decode_plan(int M, int K, int cap, DecodePlan* P) {
             size_t o = (size_t)s * kDecStageBytes;
             P->off_xq = (uint32_t)o;
             o += xq;
+            P->off_xstage = (uint32_t)o;
+            o += xstage;
             P->off_mask = (uint32_t)o;
             o += mask;
             P->off_pre = (uint32_t)o;
             o += pre;
             P->off_list = (uint32_t)o;
             o += list;
+            P->off_xo = (uint32_t)o;
+            o += xo;
+            P->off_oslot = (uint32_t)o;
+            o += oslot;
             P->off_bars = (uint32_t)align_up(o, 8);
             P->bytes = (uint32_t)total;
+            P->cluster = cluster;
             return true;
         }
+    }
+    return false;
+}
+
+// The decode plan and grid for one call: clusters of kDecCluster CTAs when
+// there are enough CTAs and the staging fits, else each CTA alone.
+bool decode_setup(int M, int K, int N, int cap, int sms, DecodePlan* P, int* splits, int* grid) {
+    const int tiles = cdiv(N, kDecTileN);
+    *splits = decode_splits(N, K, sms);
+    const int ctas = tiles * *splits;
+    if (ctas >= 2 * kDecCluster && decode_plan(M, K, cap, kDecCluster, P)) {
+        *grid = cdiv(ctas, kDecCluster) * kDecCluster;
+        return true;
+    }
+    if (decode_plan(M, K, cap, 1, P)) {
+        *grid = ctas;
+        return true;
     }
     return false;
 }
@@ -430,7 +516,7 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
     if (ws_bytes < L.total) return INT8MM_ERR_WORKSPACE_TOO_SMALL;
 
     DecodePlan dp{};
-    const bool decode_fits = decode_plan(M, K, max_outliers, &dp);
+    const bool decode_fits = decode_plan(M, K, max_outliers, 1, &dp);
     bool use_decode;
     if (path == INT8MM_PATH_DECODE) {
         if (!decode_fits) return INT8MM_ERR_INVALID_ARGUMENT;
@@ -466,6 +552,7 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
         p.K = K;
         p.N = N;
         p.thr = threshold;
+        p.thr_bits2 = fp16_threshold_bits2(threshold);
         p.cap = max_outliers;
         p.wq = w->wq;
         p.ca = w->col_absmax;
@@ -482,20 +569,25 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
         p.status = status;
         p.wait_limit_ns = wait_ns;
         p.test_flags = test_flags;
+        int splits = 1, grid = 1;
+        if (!decode_setup(M, K, N, max_outliers, info->sm_count, &dp, &splits, &grid)) return INT8MM_ERR_INVALID_ARGUMENT;
         p.num_tiles = cdiv(N, kDecTileN);
         p.kb_per_tile = cdiv(K, 128);
+        p.splits = splits;
+        p.cluster = dp.cluster;
         p.stages = dp.stages;
         p.groups = dp.groups;
         p.off_xq = dp.off_xq;
         p.off_mask = dp.off_mask;
         p.off_pre = dp.off_pre;
         p.off_list = dp.off_list;
+        p.off_xo = dp.off_xo;
+        p.off_oslot = dp.off_oslot;
         p.off_bars = dp.off_bars;
-        const long long units = (long long)p.num_tiles * p.kb_per_tile;
-        const int grid = (int)std::min<long long>(units, info->sm_count);
+        p.off_xstage = dp.off_xstage;
         cudaError_t e = timed ? cudaEventRecord(ev0, s) : cudaSuccess;
         if (e == cudaSuccess)
-            e = launch(k_decode_int8_sm100, dim3(grid), dim3(kDecThreads), dp.bytes, s, !timed, tm_w, p);
+            e = launch_ex(k_decode_int8_sm100, dim3(grid), dim3(kDecThreads), dp.bytes, s, !timed, dp.cluster, tm_w, p);
         if (e == cudaSuccess && timed) e = cudaEventRecord(ev1, s);
         return cuda_status(e);
     }
@@ -585,7 +677,7 @@ int8mm_status int8mm_forward_decode_noalloc(const uint16_t* X, int M, const int8
     if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(w->wq, 256)) return INT8MM_ERR_MISALIGNED;
     const int cap = K;
     DecodePlan dp{};
-    if (!decode_plan(M, K, cap, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!decode_plan(M, K, cap, 1, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
     const NoAllocLayout L = noalloc_layout(M, K, N);
     if (L.total > kNoAllocBytes) return INT8MM_ERR_INVALID_ARGUMENT;
 
@@ -606,6 +698,7 @@ int8mm_status int8mm_forward_decode_noalloc(const uint16_t* X, int M, const int8
     p.K = K;
     p.N = N;
     p.thr = threshold;
+    p.thr_bits2 = fp16_threshold_bits2(threshold);
     p.cap = cap;
     p.wq = w->wq;
     p.ca = w->col_absmax;
@@ -622,21 +715,26 @@ int8mm_status int8mm_forward_decode_noalloc(const uint16_t* X, int M, const int8
     p.status = reinterpret_cast<int*>(b);
     p.wait_limit_ns = kDefaultWaitNs;
     p.test_flags = 0;
+    int splits = 1, grid = 1;
+    if (!decode_setup(M, K, N, cap, info->sm_count, &dp, &splits, &grid)) return INT8MM_ERR_INVALID_ARGUMENT;
     p.num_tiles = cdiv(N, kDecTileN);
     p.kb_per_tile = cdiv(K, 128);
+    p.splits = splits;
+    p.cluster = dp.cluster;
     p.stages = dp.stages;
     p.groups = dp.groups;
     p.off_xq = dp.off_xq;
     p.off_mask = dp.off_mask;
     p.off_pre = dp.off_pre;
     p.off_list = dp.off_list;
+    p.off_xo = dp.off_xo;
+    p.off_oslot = dp.off_oslot;
     p.off_bars = dp.off_bars;
-    const long long units = (long long)p.num_tiles * p.kb_per_tile;
-    const int grid = (int)std::min<long long>(units, info->sm_count);
+    p.off_xstage = dp.off_xstage;
     // status word, count, tile counters and the partial sums start at zero
     cudaError_t e = cudaMemsetAsync(b, 0, L.clear_bytes, s);
     if (e == cudaSuccess)
-        e = launch(k_decode_int8_sm100, dim3(grid), dim3(kDecThreads), dp.bytes, s, false, tm_w, p);
+        e = launch_ex(k_decode_int8_sm100, dim3(grid), dim3(kDecThreads), dp.bytes, s, false, dp.cluster, tm_w, p);
     return cuda_status(e);
 }
 

@@ -107,6 +107,23 @@ def test_decode_path_threshold_inf_and_all_outliers():
     _run_case(4, 256, 272, 0, thr=1e-30, path="decode", keep="all", seed=13)
 
 
+@pytest.mark.parametrize("thr", [6.0, 5.998, 5.99609375, 65504.0, 70000.0])
+@pytest.mark.parametrize("path", ["decode", "gemm"])
+def test_threshold_boundaries(thr, path):
+    """Values exactly at, just below and just above the threshold (which may
+    fall between two fp16 values) are classified like the oracle does."""
+    M, K, N = 8, 512, 272
+    X, W, cols = synth.make_case(M, K, N, n_seed=0, seed=41)
+    X[1, 10] = 6.0
+    X[2, 20] = -5.99609375          # the fp16 value just below 6
+    X[3, 30] = 6.00390625           # the fp16 value just above 6
+    X[4, 40] = 65504.0
+    X[5, 50] = 60000.0
+    w = parity.gpu_prepare(W, [10, 20])
+    prep, r = parity.oracle_full(X, W, [10, 20], thr)
+    parity.check_forward_full(parity.gpu_forward(X, w, thr, path=path), r)
+
+
 def test_decode_workspace_is_reusable():
     """Split-K partial sums and tile counters return to zero after each call."""
     M, K, N = 8, 4096, 2048
