@@ -131,8 +131,10 @@ int8mm_status int8mm_forward(const uint16_t* X, int M, const int8mm_weight* w, f
 
 enum {
     INT8MM_PATH_AUTO = 0,    /* decode kernel for M <= 16, tiled GEMM otherwise */
-    INT8MM_PATH_GEMM = 1,    /* detect -> quantise -> gather -> tcgen05 GEMM, any M */
-    INT8MM_PATH_DECODE = 2   /* single fused weight-streaming kernel, M <= 16 */
+    INT8MM_PATH_GEMM = 1,    /* detect -> quantise -> gather -> tcgen05 GEMM, any M (SM-pair
+                                256 x 256 tiles when M > 128) */
+    INT8MM_PATH_DECODE = 2,  /* single fused weight-streaming kernel, M <= 16 */
+    INT8MM_PATH_GEMM_1SM = 3 /* the tiled path with single-SM 128 x 256 GEMM tiles (for tests) */
 };
 
 typedef struct {

@@ -21,14 +21,14 @@ import numpy as np
 import torch
 
 from . import _abi
-from ._abi import PATH_AUTO, PATH_DECODE, PATH_GEMM, Int8mmError
+from ._abi import PATH_AUTO, PATH_DECODE, PATH_GEMM, PATH_GEMM_1SM, Int8mmError
 
 __all__ = [
     "PreparedWeight", "Workspace", "prepare_weight", "forward", "device_status", "library",
     "Int8mmError", "PATH_AUTO", "PATH_GEMM", "PATH_DECODE",
 ]
 
-_PATHS = {"auto": PATH_AUTO, "gemm": PATH_GEMM, "decode": PATH_DECODE}
+_PATHS = {"auto": PATH_AUTO, "gemm": PATH_GEMM, "decode": PATH_DECODE, "gemm1sm": PATH_GEMM_1SM}
 
 
 def library():

@@ -22,7 +22,7 @@ STATUS_NAMES = {
     6: "INT8MM_ERR_TIMEOUT",
     7: "INT8MM_ERR_OUTLIER_OVERFLOW",
 }
-PATH_AUTO, PATH_GEMM, PATH_DECODE = 0, 1, 2
+PATH_AUTO, PATH_GEMM, PATH_DECODE, PATH_GEMM_1SM = 0, 1, 2, 3
 
 # Every symbol the header declares.
 EXPORTS = (

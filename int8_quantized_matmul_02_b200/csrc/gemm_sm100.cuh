@@ -369,6 +369,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
     }
 
+    if (threadIdx.x == 0 && *abort_flag) settle_after_abort();  // copies issued before the abort land first
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

@@ -14,6 +14,7 @@
 
 #include "int8mm.h"
 #include "decode_sm100.cuh"
+#include "gemm2sm_sm100.cuh"
 #include "gemm_sm100.cuh"
 #include "quant_kernels.cuh"
 
@@ -68,7 +69,11 @@ int8mm_status current_device(int* dev_out, DeviceInfo** info_out) {
             cudaFuncSetAttribute(k_gemm_int8_sm100<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGemmSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(k_decode_int8_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kMaxSmemOptin) != cudaSuccess) {
+                                 kMaxSmemOptin) != cudaSuccess ||
+            cudaFuncSetAttribute(k_gemm_int8_2sm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kG2SmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(k_gemm_int8_2sm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kG2SmemBytes) != cudaSuccess) {
             cudaGetLastError();
             return INT8MM_ERR_CUDA;
         }
@@ -501,7 +506,7 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
     if (!shape_ok(M, K, N) || max_outliers < 0 || max_outliers > K) return INT8MM_ERR_INVALID_ARGUMENT;
     if (!(threshold > 0.0f)) return INT8MM_ERR_INVALID_ARGUMENT;  // also rejects NaN
     const int path = opts ? opts->path : INT8MM_PATH_AUTO;
-    if (path < INT8MM_PATH_AUTO || path > INT8MM_PATH_DECODE) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (path < INT8MM_PATH_AUTO || path > INT8MM_PATH_GEMM_1SM) return INT8MM_ERR_INVALID_ARGUMENT;
     int32_t* acc_out = opts ? opts->acc_out : nullptr;
     cudaEvent_t ev0 = opts ? reinterpret_cast<cudaEvent_t>(opts->main_start_event) : nullptr;
     cudaEvent_t ev1 = opts ? reinterpret_cast<cudaEvent_t>(opts->main_stop_event) : nullptr;
@@ -521,7 +526,7 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
     if (path == INT8MM_PATH_DECODE) {
         if (!decode_fits) return INT8MM_ERR_INVALID_ARGUMENT;
         use_decode = true;
-    } else if (path == INT8MM_PATH_GEMM) {
+    } else if (path == INT8MM_PATH_GEMM || path == INT8MM_PATH_GEMM_1SM) {
         use_decode = false;
     } else {
         use_decode = decode_fits;
@@ -619,28 +624,25 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
         e = launch(k_detect, dim3(gx, gy), dim3(256), 0, s, false, X, M, K, threshold, rows, mask);
     }
     if (e == cudaSuccess) {
-        const int grid = std::min(M, sms * 8);
+        const int grid = std::max(1, std::min(cdiv(M, 8), sms * 4));
         const size_t smem = (size_t)cdiv(K, 32) * 8;
-        if (K <= 16384)
-            e = launch(k_quant_rows<true>, dim3(grid), dim3(256), smem, s, true, X, M, K, (const uint32_t*)mask,
-                       max_outliers, kp, xq, ra, xo, idx, n_out, status);
-        else
-            e = launch(k_quant_rows<false>, dim3(grid), dim3(256), smem, s, true, X, M, K, (const uint32_t*)mask,
-                       max_outliers, kp, xq, ra, xo, idx, n_out, status);
+        e = launch(k_quant_rows, dim3(grid), dim3(256), smem, s, true, X, M, K, (const uint32_t*)mask, max_outliers,
+                   kp, xq, ra, xo, idx, n_out, status);
     }
     if (e == cudaSuccess)
         e = launch(k_gather_wo, dim3(cdiv(N, 64)), dim3(256), 0, s, true, (const int8_t*)w->wq,
                    (const float*)w->col_absmax, (const uint16_t*)w->w_keep, (const int32_t*)w->keep_slot, K, N,
                    (const int32_t*)idx, (const int32_t*)n_out, max_outliers, kp, wo, mask);
     if (e == cudaSuccess) {
+        const bool pair = (path != INT8MM_PATH_GEMM_1SM) && M > kGemmBM;
         GemmParams p{};
         p.M = M;
         p.N = N;
         p.K = K;
-        p.num_m_blocks = cdiv(M, kGemmBM);
-        p.num_n_blocks = cdiv(N, kGemmBN);
+        p.num_m_blocks = cdiv(M, pair ? kG2BM : kGemmBM);
+        p.num_n_blocks = cdiv(N, pair ? kG2BN : kGemmBN);
         p.num_tiles = p.num_m_blocks * p.num_n_blocks;
-        p.group_m = std::min(16, p.num_m_blocks);
+        p.group_m = std::min(pair ? 8 : 16, p.num_m_blocks);
         p.kb_int8 = cdiv(K, 128);
         p.n_outliers = n_out;
         p.cap = max_outliers;
@@ -650,13 +652,33 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
         p.status = status;
         p.wait_limit_ns = wait_ns;
         p.test_flags = test_flags;
-        const int grid = std::min(p.num_tiles, sms);
-        if (timed) e = cudaEventRecord(ev0, s);
-        if (e == cudaSuccess)
-            e = acc_out ? launch(k_gemm_int8_sm100<true>, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, s,
-                                 !timed, tm_a, tm_b, tm_xo, tm_wo, tm_y, p)
-                        : launch(k_gemm_int8_sm100<false>, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, s,
-                                 !timed, tm_a, tm_b, tm_xo, tm_wo, tm_y, p);
+        if (pair) {
+            // each CTA of the pair loads 128 rows of B / Wo per slice
+            CUtensorMap tm_b2, tm_wo2;
+            if (!make_map(&tm_b2, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq, K, N, K, 128, 128)) return INT8MM_ERR_CUDA;
+            if (kp > 0) {
+                if (!make_map(&tm_wo2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wo, kp, N, (uint64_t)kp * 2, 64, 128))
+                    return INT8MM_ERR_CUDA;
+            } else {
+                tm_wo2 = tm_b2;
+            }
+            const int clusters = std::min(p.num_tiles, sms / 2);
+            const int grid = 2 * clusters;
+            if (timed) e = cudaEventRecord(ev0, s);
+            if (e == cudaSuccess)
+                e = acc_out ? launch_ex(k_gemm_int8_2sm<true>, dim3(grid), dim3(kGemmThreads), kG2SmemBytes, s, !timed, 2,
+                                        tm_a, tm_b2, tm_xo, tm_wo2, tm_y, p)
+                            : launch_ex(k_gemm_int8_2sm<false>, dim3(grid), dim3(kGemmThreads), kG2SmemBytes, s, !timed, 2,
+                                        tm_a, tm_b2, tm_xo, tm_wo2, tm_y, p);
+        } else {
+            const int grid = std::min(p.num_tiles, sms);
+            if (timed) e = cudaEventRecord(ev0, s);
+            if (e == cudaSuccess)
+                e = acc_out ? launch(k_gemm_int8_sm100<true>, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, s,
+                                     !timed, tm_a, tm_b, tm_xo, tm_wo, tm_y, p)
+                            : launch(k_gemm_int8_sm100<false>, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, s,
+                                     !timed, tm_a, tm_b, tm_xo, tm_wo, tm_y, p);
+        }
         if (e == cudaSuccess && timed) e = cudaEventRecord(ev1, s);
     }
     return cuda_status(e);

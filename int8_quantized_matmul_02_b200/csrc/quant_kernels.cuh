@@ -215,19 +215,20 @@ __device__ __forceinline__ uint2 quant_chunk(uint4 v, const uint32_t* smask, con
 // Xq[m,k] = outlier ? 0 : q(X[m,k]), Xo[m, slot(k)] = X[m,k] for outlier k,
 // with Xo zero-padded to a multiple of 64 columns.  Block 0 also writes the
 // ascending outlier list, the count and the overflow flag.
-// Block: 256 threads; the grid strides over rows.  kRegs: the row fits in 8
-// 16-byte chunks per thread (K <= 16384) and is read once.
-template <bool kRegs>
-__global__ void __launch_bounds__(256, 2) k_quant_rows(const uint16_t* __restrict__ X, int M, int K,
+// One warp per row (no block barrier inside the row loop): a first pass over
+// the row takes the absmax with 8 independent 16-byte loads in flight per
+// lane, a second pass (served by L1/L2) writes the codes.  Block: 256 threads
+// = 8 rows at a time; the grid strides over rows.
+__global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__ X, int M, int K,
                                                     const uint32_t* __restrict__ mask, int cap, int kp,
                                                     int8_t* __restrict__ Xq, float* __restrict__ ra,
                                                     uint16_t* __restrict__ Xo, int32_t* __restrict__ idx,
                                                     int32_t* __restrict__ n_out, int* __restrict__ status) {
     extern __shared__ uint32_t qsm[];
     const int nw = (K + 31) / 32;
-    uint32_t* smask = qsm;          // nw words
-    int* spre = reinterpret_cast<int*>(qsm + nw);  // nw exclusive prefix counts
-    __shared__ uint32_t red[8];
+    uint32_t* smask = qsm;                          // nw words
+    int* spre = reinterpret_cast<int*>(qsm + nw);   // nw exclusive prefix counts
+    __shared__ int red[8];
     __shared__ int total_sh;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
@@ -237,22 +238,23 @@ __global__ void __launch_bounds__(256, 2) k_quant_rows(const uint16_t* __restric
     // exclusive scan of popcounts over the mask words
     int carry = 0;
     for (int base = 0; base < nw; base += 256) {
-        int w = base + tid;
-        uint32_t word = w < nw ? mask[w] : 0u;
+        const int w = base + tid;
+        const uint32_t word = w < nw ? mask[w] : 0u;
         if (w < nw) smask[w] = word;
-        int c = __popc(word);
+        const int c = __popc(word);
         int incl = c;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            int v = __shfl_up_sync(0xffffffffu, incl, o);
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += v;
         }
         if (lane == 31) red[warp] = incl;
         __syncthreads();
-        int wsum = 0;
-        for (int i = 0; i < warp; ++i) wsum += red[i];
-        int blk_total = 0;
-        for (int i = 0; i < 8; ++i) blk_total += red[i];
+        int wsum = 0, blk_total = 0;
+        for (int i = 0; i < 8; ++i) {
+            if (i < warp) wsum += red[i];
+            blk_total += red[i];
+        }
         if (w < nw) spre[w] = carry + wsum + incl - c;
         carry += blk_total;
         __syncthreads();
@@ -272,7 +274,7 @@ __global__ void __launch_bounds__(256, 2) k_quant_rows(const uint16_t* __restric
             uint32_t word = smask[w];
             int s = spre[w];
             while (word) {
-                int b = __ffs(word) - 1;
+                const int b = __ffs(word) - 1;
                 idx[s++] = w * 32 + b;
                 word &= word - 1;
             }
@@ -280,46 +282,35 @@ __global__ void __launch_bounds__(256, 2) k_quant_rows(const uint16_t* __restric
     }
 
     const int nchunk = K / 8;
-    for (int m = blockIdx.x; m < M; m += gridDim.x) {
+    for (int m = blockIdx.x * 8 + warp; m < M; m += gridDim.x * 8) {
         const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)m * K);
-        uint4 regs[kRegs ? 8 : 1];
         uint32_t amax = 0;
-        if constexpr (kRegs) {
+        for (int c0 = lane; c0 < nchunk; c0 += 32 * 8) {
+            uint4 v[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int c = tid + i * 256;
-                if (c < nchunk) {
-                    regs[i] = __ldg(xr + c);
-                    amax = max(amax, chunk_inlier_absmax(regs[i], smask, c));
-                }
-            }
-        } else {
-            for (int c = tid; c < nchunk; c += 256) amax = max(amax, chunk_inlier_absmax(__ldg(xr + c), smask, c));
+            for (int i = 0; i < 8; ++i)
+                if (c0 + 32 * i < nchunk) v[i] = __ldg(xr + c0 + 32 * i);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (c0 + 32 * i < nchunk) amax = max(amax, chunk_inlier_absmax(v[i], smask, c0 + 32 * i));
         }
-        // block max
         amax = __reduce_max_sync(0xffffffffu, amax);
-        __syncthreads();
-        if (lane == 0) red[warp] = amax;
-        __syncthreads();
-        uint32_t bm = red[0];
-#pragma unroll
-        for (int i = 1; i < 8; ++i) bm = max(bm, red[i]);
-        const float rmax = half_bits_to_float(bm);
+        const float rmax = half_bits_to_float(amax);
         const float scale = rmax > 0.0f ? __fdiv_rn(127.0f, rmax) : 0.0f;
-        if (tid == 0) ra[m] = rmax;
+        if (lane == 0) ra[m] = rmax;
         uint2* qr = reinterpret_cast<uint2*>(Xq + (size_t)m * K);
         uint16_t* xo_row = Xo + (size_t)m * kp;
-        if constexpr (kRegs) {
+        for (int c0 = lane; c0 < nchunk; c0 += 32 * 8) {
+            uint4 v[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int c = tid + i * 256;
-                if (c < nchunk) qr[c] = quant_chunk(regs[i], smask, spre, c, rmax, scale, n_eff, xo_row);
-            }
-        } else {
-            for (int c = tid; c < nchunk; c += 256)
-                qr[c] = quant_chunk(__ldg(xr + c), smask, spre, c, rmax, scale, n_eff, xo_row);
+            for (int i = 0; i < 8; ++i)
+                if (c0 + 32 * i < nchunk) v[i] = __ldg(xr + c0 + 32 * i);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (c0 + 32 * i < nchunk)
+                    qr[c0 + 32 * i] = quant_chunk(v[i], smask, spre, c0 + 32 * i, rmax, scale, n_eff, xo_row);
         }
-        for (int j = n_eff + tid; j < n_pad; j += 256) xo_row[j] = 0;
+        for (int j = n_eff + lane; j < n_pad; j += 32) xo_row[j] = 0;
     }
 }
 

@@ -38,12 +38,15 @@ def _run_case(M, K, N, n_seed, thr=6.0, path="auto", keep="seeded", cap=None, se
 
 @pytest.mark.parametrize("M,K,N,n_seed", [
     (16, 256, 384, 2),        # the tiny configuration's shape
-    (300, 1040, 784, 4),      # several 128 x 256 tiles, ragged M, N and K
+    (300, 1040, 784, 4),      # several tiles, ragged M, N and K
     (129, 512, 528, 3),
     (256, 2048, 512, 7),
+    (700, 1024, 1040, 5),     # several SM-pair tiles with a ragged pair
 ])
-def test_gemm_path_matches_oracle(M, K, N, n_seed):
-    _run_case(M, K, N, n_seed, path="gemm")
+@pytest.mark.parametrize("path", ["gemm", "gemm1sm"])
+def test_gemm_path_matches_oracle(M, K, N, n_seed, path):
+    """"gemm" uses SM-pair 256 x 256 tiles for M > 128; "gemm1sm" the single-SM kernel."""
+    _run_case(M, K, N, n_seed, path=path)
 
 
 @pytest.mark.parametrize("M", [1, 8, 17, 64, 65, 129])
