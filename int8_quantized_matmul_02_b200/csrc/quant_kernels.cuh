@@ -187,6 +187,38 @@ __device__ __forceinline__ uint32_t inlier_absmax_flags(uint4 v, uint32_t fl) {
     return amax;
 }
 
+// round_half_even(x * scale) clamped to [-127, 127], with the rounding done by
+// adding 1.5 * 2^23 in fp32: for |v| < 2^22 the sum RN(v + 1.5*2^23) keeps
+// round_half_even(v) in its low mantissa bits, so the result equals
+// __float2int_rn(v) exactly (here |v| <= 127.0001) at full fp32 rate.
+__device__ __forceinline__ int quant1_fast(float x, float scale) {
+    const float r = __fadd_rn(__fmul_rn(x, scale), 12582912.0f);
+    return max(-127, min(127, __float_as_int(r) - 0x4B400000));
+}
+
+// Codes of an 8-column chunk with no outlier column (the common case).
+__device__ __forceinline__ uint2 quant8_plain(uint4 v, float scale) {
+    const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+    int q[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[j]));
+        q[2 * j] = quant1_fast(f.x, scale);
+        q[2 * j + 1] = quant1_fast(f.y, scale);
+    }
+    const uint32_t lo = __byte_perm(__byte_perm((uint32_t)q[0], (uint32_t)q[1], 0x0040),
+                                    __byte_perm((uint32_t)q[2], (uint32_t)q[3], 0x0040), 0x5410);
+    const uint32_t hi = __byte_perm(__byte_perm((uint32_t)q[4], (uint32_t)q[5], 0x0040),
+                                    __byte_perm((uint32_t)q[6], (uint32_t)q[7], 0x0040), 0x5410);
+    return make_uint2(lo, hi);
+}
+
+// Max |x| (fp16 bits) of an 8-column chunk with no outlier column.
+__device__ __forceinline__ uint32_t chunk_absmax_plain(uint4 v) {
+    const uint32_t m = __vmaxu2(__vmaxu2(abs_bits2(v.x), abs_bits2(v.y)), __vmaxu2(abs_bits2(v.z), abs_bits2(v.w)));
+    return max(m & 0xFFFFu, m >> 16);
+}
+
 // Quantise one 8-column chunk c of a row; outlier columns give 0 and are
 // copied to their slot of the row's fp16 outlier vector.
 __device__ __forceinline__ uint2 quant_chunk(uint4 v, const uint32_t* smask, const int* spre, int c, float rmax,
@@ -291,8 +323,13 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
             for (int i = 0; i < 8; ++i)
                 if (c0 + 32 * i < nchunk) v[i] = __ldg(xr + c0 + 32 * i);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (c0 + 32 * i < nchunk) amax = max(amax, chunk_inlier_absmax(v[i], smask, c0 + 32 * i));
+            for (int i = 0; i < 8; ++i) {
+                const int c = c0 + 32 * i;
+                if (c < nchunk) {
+                    const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
+                    amax = max(amax, fl ? chunk_inlier_absmax(v[i], smask, c) : chunk_absmax_plain(v[i]));
+                }
+            }
         }
         amax = __reduce_max_sync(0xffffffffu, amax);
         const float rmax = half_bits_to_float(amax);
@@ -306,9 +343,13 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
             for (int i = 0; i < 8; ++i)
                 if (c0 + 32 * i < nchunk) v[i] = __ldg(xr + c0 + 32 * i);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (c0 + 32 * i < nchunk)
-                    qr[c0 + 32 * i] = quant_chunk(v[i], smask, spre, c0 + 32 * i, rmax, scale, n_eff, xo_row);
+            for (int i = 0; i < 8; ++i) {
+                const int c = c0 + 32 * i;
+                if (c < nchunk) {
+                    const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
+                    qr[c] = fl ? quant_chunk(v[i], smask, spre, c, rmax, scale, n_eff, xo_row) : quant8_plain(v[i], scale);
+                }
+            }
         }
         for (int j = n_eff + lane; j < n_pad; j += 32) xo_row[j] = 0;
     }

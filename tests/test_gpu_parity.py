@@ -127,6 +127,31 @@ def test_threshold_boundaries(thr, path):
     parity.check_forward_full(parity.gpu_forward(X, w, thr, path=path), r)
 
 
+@pytest.mark.parametrize("amax", [5.99609375, 3.140625, 0.46044921875, 1.5947265625, 0.01229095458984375])
+@pytest.mark.parametrize("path", ["decode", "gemm"])
+def test_quantisation_rule_every_fp16_value(amax, path):
+    """Every fp16 value in [-absmax, absmax] (including those where x * scale
+    falls exactly half-way between two integers) gets the oracle's code."""
+    h = np.arange(0, 0x7C00, dtype=np.uint16).view(np.float16)
+    pos = h[h.astype(np.float64) <= amax]
+    vals = np.concatenate([pos, -pos]).astype(np.float16)
+    M, N = 16, 64  # the values spread over 16 rows, each row also holding absmax
+    per = (vals.size + M - 1) // M
+    K = (per + 1 + 15) // 16 * 16
+    X = np.zeros((M, K), dtype=np.float16)
+    for m in range(M):
+        part = vals[m * per:(m + 1) * per]
+        X[m, 0] = amax if m % 2 == 0 else -amax
+        X[m, 1:1 + part.size] = part
+    X = torch.from_numpy(X)
+    W = torch.from_numpy((np.random.default_rng(0).standard_normal((K, N)) * 0.02).astype(np.float16))
+    w = parity.gpu_prepare(W, [])
+    g = parity.gpu_forward(X, w, 6.0, path=path)
+    Xq, ra, _ = oracle.quantize_rows(X.numpy(), oracle.detect_outliers(X.numpy(), 6.0))
+    assert np.array_equal(g["ra"].view(np.uint32), ra.view(np.uint32))
+    assert np.array_equal(g["xq_dev"].cpu().numpy(), Xq)
+
+
 def test_decode_workspace_is_reusable():
     """Split-K partial sums and tile counters return to zero after each call."""
     M, K, N = 8, 4096, 2048
