@@ -130,28 +130,36 @@ class ClockSampler:
                 "samples": len(sms)}
 
 
-def kernel_source_sha() -> str:
+KERNEL_SOURCES = {
+    "k_gemm_int8_2sm": ("gemm2sm_sm100.cuh", "gemm_sm100.cuh", "sm100_ptx.cuh"),
+    "k_gemm_int8_sm100": ("gemm_sm100.cuh", "sm100_ptx.cuh"),
+    "k_decode_int8_sm100": ("decode_sm100.cuh", "quant_kernels.cuh", "sm100_ptx.cuh"),
+}
+
+
+def kernel_source_sha(kernel: str) -> str:
+    """Hash of the source files a kernel is compiled from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "int8_quantized_matmul_02_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(fh.read())
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str, workload: str, units_scale: float = 1.0):
-    """DRAM bytes per launch from a committed ncu summary, or None when the
-    kernel sources changed since the counters were taken."""
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary
+    (profiles/traffic.json), or None when the kernel's sources changed since
+    the counters were taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(f"{kernel}@{workload}")
-    if not e or e.get("source_sha") != kernel_source_sha():
+    if not e or e.get("source_sha") != kernel_source_sha(kernel):
         return None
-    return float(e["dram_bytes_per_launch"]) * units_scale
+    return float(e["dram_bytes_per_launch"])
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -477,8 +485,9 @@ def main():
 
     per_step_max, value = combine_ranks(per_step_s, value_local * per_step_s, dev, _pg is not None)
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = recorded_traffic("k_gemm_int8_sm100" if not small else "k_decode_int8_sm100", args.workload)
-    roof["kernel"] = "k_gemm_int8_sm100" if not small else "k_decode_int8_sm100"
+    kern = "k_decode_int8_sm100" if small else ("k_gemm_int8_2sm" if wl.M > 128 else "k_gemm_int8_sm100")
+    roof["traffic"] = recorded_traffic(kern, args.workload)
+    roof["kernel"] = kern
     roof["ms_per_launch"] = kern_s * 1e3
     roof["peak_source"] = pk_kind
 
