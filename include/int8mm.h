@@ -188,14 +188,11 @@ int8mm_status int8mm_get_device_status(const void* ws, void* stream, int32_t* n_
  * device-wide synchronisation of cudaMalloc are not acceptable.
  *
  * Same result as int8mm_forward on the fused decode kernel, but the scratch
- * memory (outlier list and count, status word, row absmax, int8 codes,
- * split-K partial sums and tile counters) lives in one file-scope device
- * array of INT8MM_NOALLOC_SCRATCH_BYTES inside the library, which every GPU
- * that loads the library holds until the process exits.  The caller still
- * passes X, the prepared weight and Y.
- *   Limits: 1 <= M <= 16, K <= 16384, N <= 65536, and (M, K) must fit the
- *   decode kernel's shared memory (M <= 8 with any K up to the limit;
- *   M <= 16 with K <= 8192).  Larger sizes return
+ * memory (outlier list and count, status word, row absmax, int8 codes)
+ * lives in one file-scope device array of INT8MM_NOALLOC_SCRATCH_BYTES
+ * inside the library, which every GPU that loads the library holds until the
+ * process exits.  The caller still passes X, the prepared weight and Y.
+ *   Limits: 1 <= M <= 16, K <= 16384, N <= 65536.  Larger sizes return
  *   INT8MM_ERR_INVALID_ARGUMENT and touch nothing.
  *   max_outliers is K: every detected outlier column is handled.
  * It calls no cudaMalloc, cudaFree or other allocating routine.  The first
@@ -207,7 +204,7 @@ int8mm_status int8mm_get_device_status(const void* ws, void* stream, int32_t* n_
  * the GPU (on different streams, or from different host threads) race and
  * give wrong results.  Device-side errors are read back with
  * int8mm_noalloc_device_status. */
-#define INT8MM_NOALLOC_SCRATCH_BYTES (4718592u)
+#define INT8MM_NOALLOC_SCRATCH_BYTES (524288u)
 
 int8mm_status int8mm_forward_decode_noalloc(const uint16_t* X, int M, const int8mm_weight* w,
                                             float threshold, uint16_t* Y, void* stream);

@@ -68,7 +68,9 @@ int8mm_status current_device(int* dev_out, DeviceInfo** info_out) {
                                  kGemmSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(k_gemm_int8_sm100<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGemmSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(k_decode_int8_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(k_decode_int8_sm100<8, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kMaxSmemOptin) != cudaSuccess ||
+            cudaFuncSetAttribute(k_decode_int8_sm100<16, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kMaxSmemOptin) != cudaSuccess ||
             cudaFuncSetAttribute(k_gemm_int8_2sm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kG2SmemBytes) != cudaSuccess ||
@@ -140,7 +142,7 @@ WeightLayout weight_layout(int K, int N, int n_keep) {
 }
 
 struct WsLayout {
-    size_t status, n_out, mask, idx, ra, xq, xo, wo, partial, counters, total;
+    size_t status, n_out, mask, idx, ra, xq, xo, wo, total;
     int kp;
 };
 
@@ -163,13 +165,6 @@ WsLayout ws_layout(int M, int K, int N, int max_outliers) {
     o = align_up(o + (size_t)M * L.kp * 2, 256);
     L.wo = o;
     o = align_up(o + (size_t)N * L.kp * 2, 256);
-    L.partial = o;
-    L.counters = o;
-    if (M <= kMaxDecodeRows) {
-        o = align_up(o + (size_t)kMaxDecodeRows * N * 4, 256);
-        L.counters = o;
-        o = align_up(o + (size_t)cdiv(N, kDecTileN) * 4 * 4, 256);
-    }
     L.total = o;
     return L;
 }
@@ -179,7 +174,7 @@ bool shape_ok(int M, int K, int N) {
 }
 
 // Launch with optional programmatic dependent launch (PDL) and an optional
-// thread-block cluster size along x.
+// thread-block cluster size along x (0: launched without a cluster).
 template <typename Kern, typename... Args>
 cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl, int cluster,
                       Args... args) {
@@ -195,7 +190,7 @@ cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_
         attr[n].val.programmaticStreamSerializationAllowed = 1;
         ++n;
     }
-    if (cluster > 1) {
+    if (cluster > 0) {
         attr[n].id = cudaLaunchAttributeClusterDimension;
         attr[n].val.clusterDim.x = (unsigned)cluster;
         attr[n].val.clusterDim.y = 1;
@@ -209,7 +204,7 @@ cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_
 
 template <typename Kern, typename... Args>
 cudaError_t launch(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl, Args... args) {
-    return launch_ex(kern, grid, block, smem, st, pdl, 1, args...);
+    return launch_ex(kern, grid, block, smem, st, pdl, 0, args...);
 }
 
 int8mm_status cuda_status(cudaError_t e) {
@@ -242,53 +237,61 @@ uint32_t fp16_threshold_bits2(float thr) {
     return lo | (lo << 16);
 }
 
-// K split of the decode kernel: one CTA per 128-channel tile when the tiles
-// alone fill at least half of the SMs, else enough K ranges per tile to do so.
-int decode_splits(int N, int K, int sms) {
-    const int tiles = cdiv(N, kDecTileN), kbs = cdiv(K, 128);
-    const int target = std::max(1, sms / 2);
-    return std::max(1, std::min(kbs, cdiv(target, tiles)));
-}
-
-// Shared-memory plan of the decode kernel for (M, K, cap); false if it does not fit.
+// Plan of the decode kernel: clusters of `cluster` CTAs split K (each CTA
+// one K range of the cluster's `tiles` 128-channel tiles), a TMA ring of
+// `stages` 16 KB boxes, and the shared-memory offsets.
 struct DecodePlan {
-    int stages, groups;
-    uint32_t off_xq, off_mask, off_pre, off_list, off_xo, off_oslot, off_bars, off_xstage, bytes;
-    int cluster;
+    int cluster, tiles, stages, groups, grid, mr;  // mr: rows of X per thread (8 or 16)
+    uint32_t off_xq, off_mask, off_pre, off_list, off_xo, off_oslot, off_red, off_bars, bytes;
 };
 
-// CTAs per cluster that share the decode kernel's X-side steps.
-constexpr int kDecCluster = 4;
-
-// Shared-memory plan of the decode kernel for (M, K, cap) with `cluster` CTAs
-// sharing the X-side steps (each stages its share of X); false if it does not fit.
-bool decode_plan(int M, int K, int cap, int cluster, DecodePlan* P) {
-    if (M > kMaxDecodeRows || K > 65536) return false;
+// False when (M, K, cap) does not fit the kernel: M > 16, a CTA's K range
+// wider than its X-side threads hold in registers, or shared memory.
+bool decode_plan(int M, int K, int N, int cap, int sms, DecodePlan* P) {
+    if (M < 1 || M > kMaxDecodeRows) return false;
+    const int kbt = cdiv(K, 128);
+    const int rc = M <= 8 ? 2 : 1;  // 8-column chunks per X-side thread
+    int cl = 0;
+    for (int c : {4, 8}) {
+        const int cc = std::min(c, kbt);
+        if (cdiv(kbt, cc) * 16 <= rc * kDecPro) {
+            cl = cc;
+            break;
+        }
+    }
+    if (cl == 0) return false;
+    const int tiles = cdiv(N, kDecTileN);
+    // fewest tiles per cluster that keep the grid within one wave
+    int t = cl;
+    for (int c = 1; c <= cl; ++c) {
+        if ((long long)cl * cdiv(tiles, c) <= sms) {
+            t = c;
+            break;
+        }
+    }
     const int groups = (M + 7) / 8;
-    const int kb = cdiv(K, 128);
     const int nw = cdiv(K, 32);
-    const int nchunk = K / 8;
-    const size_t xq = (size_t)(kb * groups + 1) * 1024;
+    const size_t xq = (size_t)(cdiv(kbt, cl) * groups + 1) * 1024;
     const size_t mask = align_up((size_t)nw * 4, 16);
     const size_t pre = align_up((size_t)nw * 4, 16);
     const size_t list = align_up((size_t)std::min(K, std::max(cap, 1)) * 2, 16);
     const size_t xo = (size_t)kDecSmemOutliers * 16 * 2;
     const size_t oslot = (size_t)kDecSmemOutliers * 4;
-    const int nq = cdiv(cdiv(nchunk, 4), cluster) * 4;
-    const size_t xstage = cluster > 1 ? align_up((size_t)M * nq * 16, 128) : 0;
-    const size_t fixed = xq + mask + pre + list + xo + oslot + xstage;
-    const int min_stages = cluster > 1 ? 6 : 3;
-    for (int s = 16; s >= min_stages; --s) {
-        const size_t bars = (size_t)(2 * s + 6) * 8 + 256;
+    const size_t red = (size_t)16 * kDecTileN * 4;
+    const size_t fixed = xq + mask + pre + list + xo + oslot + red;
+    for (int s = 16; s >= 4; --s) {
+        const size_t bars = (size_t)(2 * s + 5) * 8 + 256;
         const size_t total = 1024 + (size_t)s * kDecStageBytes + fixed + bars;
         if (total <= (size_t)kMaxSmemOptin) {
+            P->cluster = cl;
+            P->tiles = t;
             P->stages = s;
             P->groups = groups;
+            P->grid = cl * cdiv(tiles, t);
+            P->mr = M <= 8 ? 8 : 16;
             size_t o = (size_t)s * kDecStageBytes;
             P->off_xq = (uint32_t)o;
             o += xq;
-            P->off_xstage = (uint32_t)o;
-            o += xstage;
             P->off_mask = (uint32_t)o;
             o += mask;
             P->off_pre = (uint32_t)o;
@@ -299,30 +302,53 @@ bool decode_plan(int M, int K, int cap, int cluster, DecodePlan* P) {
             o += xo;
             P->off_oslot = (uint32_t)o;
             o += oslot;
+            P->off_red = (uint32_t)o;
+            o += red;
             P->off_bars = (uint32_t)align_up(o, 8);
             P->bytes = (uint32_t)total;
-            P->cluster = cluster;
             return true;
         }
     }
     return false;
 }
 
-// The decode plan and grid for one call: clusters of kDecCluster CTAs when
-// there are enough CTAs and the staging fits, else each CTA alone.
-bool decode_setup(int M, int K, int N, int cap, int sms, DecodePlan* P, int* splits, int* grid) {
-    const int tiles = cdiv(N, kDecTileN);
-    *splits = decode_splits(N, K, sms);
-    const int ctas = tiles * *splits;
-    if (ctas >= 2 * kDecCluster && decode_plan(M, K, cap, kDecCluster, P)) {
-        *grid = cdiv(ctas, kDecCluster) * kDecCluster;
-        return true;
-    }
-    if (decode_plan(M, K, cap, 1, P)) {
-        *grid = ctas;
-        return true;
-    }
-    return false;
+// Parameters of one decode launch (the workspace pointers are the caller's).
+DecodeParams decode_params(const uint16_t* X, int M, const int8mm_weight* w, float threshold, int cap, uint16_t* Y,
+                           const DecodePlan& dp) {
+    DecodeParams p{};
+    p.X = X;
+    p.M = M;
+    p.K = w->K;
+    p.N = w->N;
+    p.thr_bits2 = fp16_threshold_bits2(threshold);
+    p.cap = cap;
+    p.wq = w->wq;
+    p.ca = w->col_absmax;
+    p.w_keep = w->w_keep;
+    p.keep_slot = w->keep_slot;
+    p.Y = Y;
+    p.num_tiles = cdiv(w->N, kDecTileN);
+    p.kb_total = cdiv(w->K, 128);
+    p.cluster = dp.cluster;
+    p.tiles_per_cluster = dp.tiles;
+    p.stages = dp.stages;
+    p.groups = dp.groups;
+    p.off_xq = dp.off_xq;
+    p.off_mask = dp.off_mask;
+    p.off_pre = dp.off_pre;
+    p.off_list = dp.off_list;
+    p.off_xo = dp.off_xo;
+    p.off_oslot = dp.off_oslot;
+    p.off_red = dp.off_red;
+    p.off_bars = dp.off_bars;
+    return p;
+}
+
+cudaError_t launch_decode(const DecodePlan& dp, const CUtensorMap& tm_w, const DecodeParams& p, cudaStream_t s,
+                          bool pdl) {
+    if (dp.mr == 8)
+        return launch_ex(k_decode_int8_sm100<8, 2>, dim3(dp.grid), dim3(kDecThreads), dp.bytes, s, pdl, dp.cluster, tm_w, p);
+    return launch_ex(k_decode_int8_sm100<16, 1>, dim3(dp.grid), dim3(kDecThreads), dp.bytes, s, pdl, dp.cluster, tm_w, p);
 }
 
 // ------------------------------------------------------------------ no-allocation decode forward
@@ -334,19 +360,15 @@ constexpr int kNoAllocMaxK = 16384;
 constexpr int kNoAllocMaxN = 65536;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocBytes];
 
-// Layout inside the array: [status, count | counters | partial sums] (the
-// part cleared before every call), then the outlier list, ra and Xq.
+// Layout inside the array: [status, count] (the part cleared before every
+// call), then the outlier list, ra and Xq.
 struct NoAllocLayout {
-    size_t counters, partial, clear_bytes, idx, ra, xq, total;
+    size_t clear_bytes, idx, ra, xq, total;
 };
 
-NoAllocLayout noalloc_layout(int M, int K, int N) {
+NoAllocLayout noalloc_layout(int M, int K) {
     NoAllocLayout L{};
     size_t o = 256;
-    L.counters = o;
-    o = align_up(o + (size_t)cdiv(N, kDecTileN) * 4 * 4, 256);
-    L.partial = o;
-    o = align_up(o + (size_t)M * N * 4, 256);
     L.clear_bytes = o;
     L.idx = o;
     o = align_up(o + (size_t)K * 4, 256);
@@ -520,8 +542,9 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
     const WsLayout L = ws_layout(M, K, N, max_outliers);
     if (ws_bytes < L.total) return INT8MM_ERR_WORKSPACE_TOO_SMALL;
 
+    // whether the decode kernel fits does not depend on the device; its grid does
     DecodePlan dp{};
-    const bool decode_fits = decode_plan(M, K, max_outliers, 1, &dp);
+    const bool decode_fits = decode_plan(M, K, N, max_outliers, 1 << 20, &dp);
     bool use_decode;
     if (path == INT8MM_PATH_DECODE) {
         if (!decode_fits) return INT8MM_ERR_INVALID_ARGUMENT;
@@ -531,11 +554,12 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
     } else {
         use_decode = decode_fits;
     }
-
     int dev;
     DeviceInfo* info;
     int8mm_status st = current_device(&dev, &info);
     if (st != INT8MM_OK) return st;
+    if (use_decode && !decode_plan(M, K, N, max_outliers, info->sm_count, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
+
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* b = static_cast<uint8_t*>(ws);
     int* status = reinterpret_cast<int*>(b + L.status);
@@ -551,21 +575,7 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
         CUtensorMap tm_w;
         if (!make_map(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq, K, N, K, 128, kDecTileN))
             return INT8MM_ERR_CUDA;
-        DecodeParams p{};
-        p.X = X;
-        p.M = M;
-        p.K = K;
-        p.N = N;
-        p.thr = threshold;
-        p.thr_bits2 = fp16_threshold_bits2(threshold);
-        p.cap = max_outliers;
-        p.wq = w->wq;
-        p.ca = w->col_absmax;
-        p.w_keep = w->w_keep;
-        p.keep_slot = w->keep_slot;
-        p.Y = Y;
-        p.partial = reinterpret_cast<int32_t*>(b + L.partial);
-        p.counters = reinterpret_cast<int32_t*>(b + L.counters);
+        DecodeParams p = decode_params(X, M, w, threshold, max_outliers, Y, dp);
         p.acc_out = acc_out;
         p.idx_out = idx;
         p.n_out = n_out;
@@ -574,25 +584,8 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
         p.status = status;
         p.wait_limit_ns = wait_ns;
         p.test_flags = test_flags;
-        int splits = 1, grid = 1;
-        if (!decode_setup(M, K, N, max_outliers, info->sm_count, &dp, &splits, &grid)) return INT8MM_ERR_INVALID_ARGUMENT;
-        p.num_tiles = cdiv(N, kDecTileN);
-        p.kb_per_tile = cdiv(K, 128);
-        p.splits = splits;
-        p.cluster = dp.cluster;
-        p.stages = dp.stages;
-        p.groups = dp.groups;
-        p.off_xq = dp.off_xq;
-        p.off_mask = dp.off_mask;
-        p.off_pre = dp.off_pre;
-        p.off_list = dp.off_list;
-        p.off_xo = dp.off_xo;
-        p.off_oslot = dp.off_oslot;
-        p.off_bars = dp.off_bars;
-        p.off_xstage = dp.off_xstage;
         cudaError_t e = timed ? cudaEventRecord(ev0, s) : cudaSuccess;
-        if (e == cudaSuccess)
-            e = launch_ex(k_decode_int8_sm100, dim3(grid), dim3(kDecThreads), dp.bytes, s, !timed, dp.cluster, tm_w, p);
+        if (e == cudaSuccess) e = launch_decode(dp, tm_w, p, s, !timed);
         if (e == cudaSuccess && timed) e = cudaEventRecord(ev1, s);
         return cuda_status(e);
     }
@@ -698,15 +691,16 @@ int8mm_status int8mm_forward_decode_noalloc(const uint16_t* X, int M, const int8
     if (!(threshold > 0.0f)) return INT8MM_ERR_INVALID_ARGUMENT;
     if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(w->wq, 256)) return INT8MM_ERR_MISALIGNED;
     const int cap = K;
-    DecodePlan dp{};
-    if (!decode_plan(M, K, cap, 1, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
-    const NoAllocLayout L = noalloc_layout(M, K, N);
+    const NoAllocLayout L = noalloc_layout(M, K);
     if (L.total > kNoAllocBytes) return INT8MM_ERR_INVALID_ARGUMENT;
+    DecodePlan dp{};
+    if (!decode_plan(M, K, N, cap, 1 << 20, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
 
     int dev;
     DeviceInfo* info;
     int8mm_status st = current_device(&dev, &info);
     if (st != INT8MM_OK) return st;
+    if (!decode_plan(M, K, N, cap, info->sm_count, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
     uint8_t* b = nullptr;
     st = noalloc_scratch(dev, &b);
     if (st != INT8MM_OK) return st;
@@ -714,21 +708,7 @@ int8mm_status int8mm_forward_decode_noalloc(const uint16_t* X, int M, const int8
 
     CUtensorMap tm_w;
     if (!make_map(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq, K, N, K, 128, kDecTileN)) return INT8MM_ERR_CUDA;
-    DecodeParams p{};
-    p.X = X;
-    p.M = M;
-    p.K = K;
-    p.N = N;
-    p.thr = threshold;
-    p.thr_bits2 = fp16_threshold_bits2(threshold);
-    p.cap = cap;
-    p.wq = w->wq;
-    p.ca = w->col_absmax;
-    p.w_keep = w->w_keep;
-    p.keep_slot = w->keep_slot;
-    p.Y = Y;
-    p.partial = reinterpret_cast<int32_t*>(b + L.partial);
-    p.counters = reinterpret_cast<int32_t*>(b + L.counters);
+    DecodeParams p = decode_params(X, M, w, threshold, cap, Y, dp);
     p.acc_out = nullptr;
     p.idx_out = reinterpret_cast<int32_t*>(b + L.idx);
     p.n_out = reinterpret_cast<int32_t*>(b + 4);
@@ -737,26 +717,9 @@ int8mm_status int8mm_forward_decode_noalloc(const uint16_t* X, int M, const int8
     p.status = reinterpret_cast<int*>(b);
     p.wait_limit_ns = kDefaultWaitNs;
     p.test_flags = 0;
-    int splits = 1, grid = 1;
-    if (!decode_setup(M, K, N, cap, info->sm_count, &dp, &splits, &grid)) return INT8MM_ERR_INVALID_ARGUMENT;
-    p.num_tiles = cdiv(N, kDecTileN);
-    p.kb_per_tile = cdiv(K, 128);
-    p.splits = splits;
-    p.cluster = dp.cluster;
-    p.stages = dp.stages;
-    p.groups = dp.groups;
-    p.off_xq = dp.off_xq;
-    p.off_mask = dp.off_mask;
-    p.off_pre = dp.off_pre;
-    p.off_list = dp.off_list;
-    p.off_xo = dp.off_xo;
-    p.off_oslot = dp.off_oslot;
-    p.off_bars = dp.off_bars;
-    p.off_xstage = dp.off_xstage;
-    // status word, count, tile counters and the partial sums start at zero
+    // the status word and the outlier count start at zero
     cudaError_t e = cudaMemsetAsync(b, 0, L.clear_bytes, s);
-    if (e == cudaSuccess)
-        e = launch_ex(k_decode_int8_sm100, dim3(grid), dim3(kDecThreads), dp.bytes, s, false, dp.cluster, tm_w, p);
+    if (e == cudaSuccess) e = launch_decode(dp, tm_w, p, s, false);
     return cuda_status(e);
 }
 

@@ -197,6 +197,11 @@ __device__ __forceinline__ void atom_max_cluster_u32(uint32_t addr, uint32_t v) 
     asm volatile("atom.shared::cluster.max.u32 _, [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
+// Relaxed atomic add (no return) on a 32-bit word of any CTA of the cluster.
+__device__ __forceinline__ void red_add_cluster_u32(uint32_t addr, uint32_t v) {
+    asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 // Arrive (release at cluster scope) on an mbarrier of any CTA of the cluster.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");

@@ -60,8 +60,8 @@ def test_workspace_bytes_rules(lib):
     assert lib.int8mm_workspace_bytes(0, 256, 384, 0) == 0
     assert lib.int8mm_workspace_bytes(16, 256, 384, 257) == 0
     assert lib.int8mm_workspace_bytes(16, 256, 384, -1) == 0
-    # decode-sized M carries the split-K partial sums, large M does not
-    assert lib.int8mm_workspace_bytes(16, 256, 384, 0) > lib.int8mm_workspace_bytes(17, 256, 384, 0) - 17 * 256
+    # the row-sized parts (codes, scales, fp16 outlier rows) grow with M
+    assert lib.int8mm_workspace_bytes(4096, 256, 384, 64) > lib.int8mm_workspace_bytes(16, 256, 384, 64)
 
 
 FAKE = 0x7F0000000000  # never dereferenced: every call below fails its argument checks first
