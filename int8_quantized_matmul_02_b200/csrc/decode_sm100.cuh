@@ -12,9 +12,10 @@
 // only its K range of X, so the outlier flags of those columns are final at
 // once (all M rows of a column are in the same CTA), quantises only those
 // columns, and shares with its peers just the flag words and the row maxima
-// (distributed shared memory, one exchange).  The int32 partial sums of a
-// tile meet in the shared memory of the tile's owner (CTA j owns tile j)
-// through cluster-scope atomic adds, exact in any order.
+// (one exchange of asynchronous stores into the peers' shared memory, which
+// complete on the receiver's mbarrier).  The int32 partial sums of a tile go
+// the same way to the tile's owner (CTA j owns tile j), one slot per source
+// CTA, and the owner adds the slots (exact in any order).
 //
 // Warp roles (384 threads):
 //   warp 0: TMA producer of 128 (channels) x 128 (K) int8 weight boxes;
@@ -144,9 +145,9 @@ __device__ __forceinline__ uint32_t chunk_flags(const uint32_t (&mx)[4], uint32_
     return fl;
 }
 
-// kMR: rows of X held in registers (8 or 16, >= M); kRC: 8-column chunks per
-// X-side thread (the CTA's K range has at most kRC * kDecPro chunks).
-template <int kMR, int kRC>
+// kR: rows per 8-column chunk group (8 or 16, >= M); kP: (chunk, row) pairs
+// per X-side thread (the CTA's K range has at most kP * kDecPro / kR chunks).
+template <int kR, int kP>
 __global__ void __launch_bounds__(kDecThreads, 1)
     k_decode_int8_sm100(const __grid_constant__ CUtensorMap tm_w, const DecodeParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -158,21 +159,20 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     uint16_t* slist = reinterpret_cast<uint16_t*>(smem + p.off_list);
     uint16_t* sxo = reinterpret_cast<uint16_t*>(smem + p.off_xo);  // [kDecSmemOutliers][16] fp16 x values
     int* soslot = reinterpret_cast<int*>(smem + p.off_oslot);      // [kDecSmemOutliers] kept-row slot
-    uint32_t* sred = reinterpret_cast<uint32_t*>(smem + p.off_red);  // [16][128] int32 sums of the owned tile
+    uint32_t* sred = reinterpret_cast<uint32_t*>(smem + p.off_red);  // [CL][128][RS] partial sums of the owned tile
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bars);
     uint64_t* full = bars;
     uint64_t* empty = bars + p.stages;
     uint64_t* tfull = bars + 2 * p.stages;
     uint64_t* xq_ready = tfull + 1;
     uint64_t* drain = tfull + 2;
-    uint64_t* xchg = tfull + 3;      // flag words and row maxima of every peer have arrived
-    uint64_t* red_done = tfull + 4;  // every peer's partial sums have arrived
+    uint64_t* xchg = tfull + 3;      // flag words and row maxima of every peer have arrived (tx bytes)
+    uint64_t* red_done = tfull + 4;  // every peer's partial sums have arrived (tx bytes)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 5);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     unsigned* sra_bits = reinterpret_cast<unsigned*>(tmem_slot + 2);  // [16] row absmax (fp16 bits)
     int* sflag = reinterpret_cast<int*>(tmem_slot + 18);              // [1] total outliers
-    float* sscale = reinterpret_cast<float*>(tmem_slot + 20);         // [16] 127 / ra
-    float* srs = reinterpret_cast<float*>(tmem_slot + 36);            // [16] ra / 127^2
+    float* srs = reinterpret_cast<float*>(tmem_slot + 20);            // [16] ra / 127^2
     const uint16_t* __restrict__ Xg = p.X;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -180,6 +180,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const int nw = (K + 31) / 32;
     const int nchunk = K / 8;
     const int CL = p.cluster;
+    const int RS = 8 * p.groups;  // rows of one partial-sum slot
     WaitCtx wctx{abort_flag, p.status, p.wait_limit_ns};
 
     // this CTA: K blocks [kb_lo, kb_hi) of tiles [tile0, tile0 + nt); it owns
@@ -203,11 +204,22 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         mbar_init(tfull, 1);
         mbar_init(xq_ready, 1);
         mbar_init(drain, 1);
-        mbar_init(xchg, CL);
-        mbar_init(red_done, CL);
+        mbar_init(xchg, 1);
+        mbar_init(red_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_w);
+        // bytes the peers will store: their flag words and M row maxima each,
+        // and (owner) one partial-sum slot per CTA of the cluster
+        uint32_t xb = 0;
+        for (int q = 0; q < CL; ++q) {
+            if (q == rank) continue;
+            const int qlo = (int)((long long)p.kb_total * q / CL), qhi = (int)((long long)p.kb_total * (q + 1) / CL);
+            xb += (uint32_t)(((min(nchunk, qhi * 16) + 3) / 4 - qlo * 4) * 4 + M * 4);
+        }
+        if (xb) mbar_arrive_expect_tx(xchg, xb);
+        else mbar_arrive(xchg);
+        if (owner && has_acc) mbar_arrive_expect_tx(red_done, (uint32_t)(CL * kDecTileN * RS * 4));
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, tmem_cols);
@@ -215,11 +227,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     if (threadIdx.x < 16) sra_bits[threadIdx.x] = 0u;
     for (int w = threadIdx.x; w < nw; w += kDecThreads) smask[w] = 0u;
-    for (int i = threadIdx.x; i < 16 * kDecTileN; i += kDecThreads) sred[i] = 0u;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    cluster_sync_all();  // every peer's barriers and buffers are initialised
+    // Peers write into this CTA's barriers and buffers only after the cluster
+    // barrier completes; each thread arrives here and waits just before its
+    // first access to a peer (the weight stream needs no peer).
+    cluster_arrive();
     const uint32_t tmem_base = *tmem_slot;
     pdl_launch_dependents();
 
@@ -252,25 +266,34 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (elect_one() && has_acc) {
+            // One thread issues every MMA, so the loop keeps its per-stage work
+            // small: descriptors are the base descriptors plus the operand
+            // offset >> 4 (the start-address field holds address >> 4 in 14
+            // bits, and shared-memory addresses stay below 2^18, so the sum
+            // never carries out of the field); 32 bytes of K are +2.
             const uint32_t idesc = idesc_s8_s32(128, 16);
-            const uint32_t sxq_addr = smem_u32(sxq);
+            const uint64_t da0 = sdesc_k128sw(smem_u32(ring));
+            const uint64_t db0 = sdesc_k128sw(smem_u32(sxq));
+            const uint64_t db_step = (uint64_t)((p.groups * 1024) >> 4);
             int stage = 0;
             uint32_t phase = 0;
             bool issued = false, ok = wait_bounded(xq_ready, 0, wctx);
             tc_fence_after();
             for (int j = 0; ok && j < nt; ++j) {
+                const uint32_t dtm = tmem_base + (uint32_t)(32 * j);
+                uint64_t db = db0;
                 for (int kb = kb_lo; kb < kb_hi; ++kb) {
-                    if (!wait_bounded(&full[stage], phase, wctx)) {
+                    if (!mbar_try_wait(&full[stage], phase) && !wait_bounded(&full[stage], phase, wctx)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = smem_u32(ring + stage * kDecStageBytes);
-                    const uint32_t sb = sxq_addr + (uint32_t)((kb - kb_lo) * p.groups * 1024);
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj)
-                        mma_s8(tmem_base + (uint32_t)(32 * j), sdesc_k128sw(sa + 32 * jj), sdesc_k128sw(sb + 32 * jj), idesc,
-                               (kb != kb_lo || jj != 0) ? 1u : 0u);
+                    const uint64_t da = da0 + (uint64_t)(stage * (kDecStageBytes >> 4));
+                    mma_s8(dtm, da, db, idesc, kb != kb_lo ? 1u : 0u);
+                    mma_s8(dtm, da + 2, db + 2, idesc, 1u);
+                    mma_s8(dtm, da + 4, db + 4, idesc, 1u);
+                    mma_s8(dtm, da + 6, db + 6, idesc, 1u);
+                    db += db_step;
                     issued = true;
                     tc_commit(&empty[stage]);
                     if (++stage == p.stages) {
@@ -289,95 +312,83 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         // ------------------------------------------------ X-side steps (warps 2..11)
         const int pt = threadIdx.x - 64;  // 0 .. kDecPro-1
         pdl_wait();                       // X belongs to earlier work on the stream
-        // (a) every chunk of this thread, all rows, in registers: the outlier
-        // flags of a chunk are final at once, and the codes come from the same
-        // registers
-        uint4 xv[kRC][kMR];
-        uint32_t cfl[kRC];
+        // (a) Thread pairs (8-column chunk, row): the kR rows of a chunk sit in
+        // kR consecutive lanes, so a chunk's outlier flags are the OR of its
+        // lanes' flags (shuffles), and a thread's row is the same for all its
+        // pairs (kDecPro is a multiple of 32 and of kR), so one running max
+        // and one scale per thread.  The values stay in registers for (b).
+        const int prow = lane % kR;
+        const bool row_ok = prow < M;
+        uint4 xv[kP];
+        uint32_t cfl[kP];
+#pragma unroll
+        for (int i = 0; i < kP; ++i) {
+            const int c = c0 + (pt + i * kDecPro) / kR;
+            if (row_ok && c < c1) xv[i] = __ldg(reinterpret_cast<const uint4*>(Xg + (size_t)prow * K) + c);
+        }
         {
+            uint32_t rmax = 0;
 #pragma unroll
-            for (int i = 0; i < kRC; ++i) {
-                const int c = c0 + pt + i * kDecPro;
-                cfl[i] = 0u;
-#pragma unroll
-                for (int m = 0; m < kMR; ++m)
-                    if (c < c1 && m < M) xv[i][m] = __ldg(reinterpret_cast<const uint4*>(Xg + (size_t)m * K) + c);
-            }
-            uint32_t rmax[kMR];
-#pragma unroll
-            for (int m = 0; m < kMR; ++m) rmax[m] = 0;
-#pragma unroll
-            for (int i = 0; i < kRC; ++i) {
-                const int c = c0 + pt + i * kDecPro;
-                if (c < c1) {
-                    uint32_t mx[4] = {0, 0, 0, 0};
-#pragma unroll
-                    for (int m = 0; m < kMR; ++m) {
-                        if (m < M) {
-                            mx[0] = __vmaxu2(mx[0], abs_bits2(xv[i][m].x));
-                            mx[1] = __vmaxu2(mx[1], abs_bits2(xv[i][m].y));
-                            mx[2] = __vmaxu2(mx[2], abs_bits2(xv[i][m].z));
-                            mx[3] = __vmaxu2(mx[3], abs_bits2(xv[i][m].w));
-                        }
-                    }
-                    const uint32_t fl = chunk_flags(mx, p.thr_bits2);
-                    cfl[i] = fl;
-                    if (fl) atomicOr(&smask[c >> 2], fl << ((c & 3) * 8));
-#pragma unroll
-                    for (int m = 0; m < kMR; ++m)
-                        if (m < M) rmax[m] = max(rmax[m], inlier_absmax_simd(xv[i][m], fl));
+            for (int i = 0; i < kP; ++i) {
+                const int c = c0 + (pt + i * kDecPro) / kR;
+                const bool ok = row_ok && c < c1;
+                uint32_t fl = 0;
+                if (ok) {
+                    const uint32_t mx[4] = {abs_bits2(xv[i].x), abs_bits2(xv[i].y), abs_bits2(xv[i].z),
+                                            abs_bits2(xv[i].w)};
+                    fl = chunk_flags(mx, p.thr_bits2);
                 }
+#pragma unroll
+                for (int off = 1; off < kR; off <<= 1) fl |= __shfl_xor_sync(0xffffffffu, fl, off);
+                cfl[i] = fl;
+                if (prow == 0 && c < c1 && fl) atomicOr(&smask[c >> 2], fl << ((c & 3) * 8));
+                if (ok) rmax = max(rmax, inlier_absmax_simd(xv[i], fl));
             }
 #pragma unroll
-            for (int m = 0; m < kMR; ++m) {
-                if (m < M) {
-                    const uint32_t r = __reduce_max_sync(0xffffffffu, rmax[m]);
-                    if (lane == 0 && r) atomicMax(&sra_bits[m], r);
-                }
-            }
+            for (int off = kR; off < 32; off <<= 1) rmax = max(rmax, __shfl_xor_sync(0xffffffffu, rmax, off));
+            if (lane < kR && row_ok && rmax) atomicMax(&sra_bits[prow], rmax);
         }
         named_bar_sync(1, kDecPro);
-        // share this CTA's flag words (its K range covers whole words) and row
-        // maxima with the peers, then wait for theirs
+        // this CTA's flag words (its K range covers whole words) and row
+        // maxima to every peer; the peers' arrive the same way
         if (CL > 1) {
+            cluster_wait();  // every peer's barriers and buffers are initialised
             for (int w = c0 / 4 + pt; w < (c1 + 3) / 4; w += kDecPro) {
                 const uint32_t val = smask[w];
-                if (val)
-                    for (int r = 0; r < CL; ++r)
-                        if (r != rank) st_cluster_u32(map_to_rank(&smask[w], r), val);
+                for (int q = 0; q < CL; ++q)
+                    if (q != rank) st_async_u32(map_to_rank(&smask[w], (uint32_t)q), val, map_to_rank(xchg, (uint32_t)q));
             }
-            if (pt < M && sra_bits[pt])
-                for (int r = 0; r < CL; ++r)
-                    if (r != rank) atom_max_cluster_u32(map_to_rank(&sra_bits[pt], r), sra_bits[pt]);
-            fence_acq_rel_cluster();
+            if (pt >= kDecPro - 16 && pt - (kDecPro - 16) < M) {
+                const int m = pt - (kDecPro - 16);
+                const uint32_t val = sra_bits[m];
+                for (int q = 0; q < CL; ++q)
+                    if (q != rank)
+                        red_async_max_u32(map_to_rank(&sra_bits[m], (uint32_t)q), val, map_to_rank(xchg, (uint32_t)q));
+            }
+        } else {
+            cluster_wait();
         }
-        named_bar_sync(1, kDecPro);
-        if (pt == 0)
-            for (int r = 0; r < CL; ++r) mbar_arrive_cluster(map_to_rank(xchg, r));
-        wait_bounded_cluster(xchg, 0, wctx);
-        // the whole mask and the row maxima are here: scales, then the codes
-        if (warp == 3 && lane < 16) {
-            const float rmax = half_bits_to_float(sra_bits[lane]);
-            sscale[lane] = rmax > 0.0f ? __fdiv_rn(127.0f, rmax) : 0.0f;
-            srs[lane] = __fdiv_rn(rmax, 16129.0f);
-            if (blockIdx.x == 0 && lane < M) p.ra_out[lane] = rmax;
-        }
-        named_bar_sync(1, kDecPro);
-        // (b) int8 codes of this CTA's K range into the shared B operand; the
+        wait_bounded(xchg, 0, wctx);
+        // the whole mask and the row maxima are here: this thread's scale,
+        // then (b) the int8 codes of its pairs into the shared B operand; the
         // first cluster also writes them to the workspace
+        {
+            const float rmax = row_ok ? half_bits_to_float(sra_bits[prow]) : 0.0f;
+            const float scl = rmax > 0.0f ? __fdiv_rn(127.0f, rmax) : 0.0f;
 #pragma unroll
-        for (int i = 0; i < kRC; ++i) {
-            const int c = c0 + pt + i * kDecPro;
-            if (c < c1) {
-#pragma unroll
-                for (int m = 0; m < kMR; ++m) {
-                    if (m < M) {
-                        const uint2 q = dec_quant8(xv[i][m], cfl[i], sscale[m]);
-                        *reinterpret_cast<uint2*>(sxq + dec_xq_off(m, (c - c0) * 8, p.groups)) = q;
-                        if ((int)blockIdx.x < CL) *reinterpret_cast<uint2*>(p.xq_out + (size_t)m * K + (size_t)c * 8) = q;
-                    }
+            for (int i = 0; i < kP; ++i) {
+                const int c = c0 + (pt + i * kDecPro) / kR;
+                if (row_ok && c < c1) {
+                    const uint2 q = dec_quant8(xv[i], cfl[i], scl);
+                    *reinterpret_cast<uint2*>(sxq + dec_xq_off(prow, (c - c0) * 8, p.groups)) = q;
+                    if ((int)blockIdx.x < CL) *reinterpret_cast<uint2*>(p.xq_out + (size_t)prow * K + (size_t)c * 8) = q;
                 }
             }
+        }
+        if (warp == 3 && lane < 16) {
+            const float rmax = half_bits_to_float(sra_bits[lane]);
+            srs[lane] = __fdiv_rn(rmax, 16129.0f);
+            if (blockIdx.x == 0 && lane < M) p.ra_out[lane] = rmax;
         }
         fence_proxy_async_smem();
         named_bar_sync(1, kDecPro);
@@ -473,27 +484,46 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                         if (m < M) o[m] = fmaf(half_bits_to_float(Xg[(size_t)m * K + k]), w, o[m]);
                 }
             }
-            // partial sums of every tile of this CTA into the owner's buffer
+            // partial sums of every tile of this CTA into this CTA's slot of the
+            // tile owner's buffer (16-byte asynchronous stores, rows of one
+            // channel together), completing on the owner's barrier
             if (has_acc && __all_sync(0xffffffffu, wait_bounded(tfull, 0, wctx))) {
                 tc_fence_after();
                 for (int j = 0; j < nt; ++j) {
                     uint32_t r[16];
                     tmem_ld16(tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(32 * j), r);
                     tmem_wait_ld();
-#pragma unroll
-                    for (int m = 0; m < 16; ++m)
-                        if (m < M) red_add_cluster_u32(map_to_rank(&sred[m * kDecTileN + ch], (uint32_t)j), r[m]);
+                    const uint32_t dst = map_to_rank(&sred[(size_t)(rank * kDecTileN + ch) * RS], (uint32_t)j);
+                    const uint32_t mb = map_to_rank(red_done, (uint32_t)j);
+                    st_async_v4(dst, r[0], r[1], r[2], r[3], mb);
+                    st_async_v4(dst + 16, r[4], r[5], r[6], r[7], mb);
+                    if (RS == 16) {
+                        st_async_v4(dst + 32, r[8], r[9], r[10], r[11], mb);
+                        st_async_v4(dst + 48, r[12], r[13], r[14], r[15], mb);
+                    }
                 }
             }
-            fence_acq_rel_cluster();
-            named_bar_sync(2, 128);
-            if (warp == 4 && lane == 0)
-                for (int r = 0; r < CL; ++r) mbar_arrive_cluster(map_to_rank(red_done, r));
-            if (owner && __all_sync(0xffffffffu, wait_bounded_cluster(red_done, 0, wctx)) && n < N) {
+            if (owner && has_acc && __all_sync(0xffffffffu, wait_bounded(red_done, 0, wctx)) && n < N) {
+                uint32_t sum[16];
+#pragma unroll
+                for (int m = 0; m < 16; ++m) sum[m] = 0u;
+                for (int q = 0; q < CL; ++q) {
+                    const uint4* src = reinterpret_cast<const uint4*>(&sred[(size_t)(q * kDecTileN + ch) * RS]);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        if (4 * v < RS) {
+                            const uint4 t = src[v];
+                            sum[4 * v] += t.x;
+                            sum[4 * v + 1] += t.y;
+                            sum[4 * v + 2] += t.z;
+                            sum[4 * v + 3] += t.w;
+                        }
+                    }
+                }
 #pragma unroll
                 for (int m = 0; m < 16; ++m) {
                     if (m < M) {
-                        const int32_t acc = (int32_t)sred[m * kDecTileN + ch];
+                        const int32_t acc = (int32_t)sum[m];
                         const float y = (float)acc * srs[m] * cav + o[m];
                         p.Y[(size_t)m * N + n] = __half_as_ushort(__float2half_rn(y));
                         if (p.acc_out) p.acc_out[(size_t)m * N + n] = acc;
@@ -503,6 +533,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         }
     }
 
+    if (warp < 2) cluster_wait();  // the X-side warps waited before their first peer access
+    // after a timeout a peer's store may still be on its way here: let it land
+    if (*abort_flag) settle_after_abort();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

@@ -68,9 +68,9 @@ int8mm_status current_device(int* dev_out, DeviceInfo** info_out) {
                                  kGemmSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(k_gemm_int8_sm100<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGemmSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(k_decode_int8_sm100<8, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(k_decode_int8_sm100<8, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kMaxSmemOptin) != cudaSuccess ||
-            cudaFuncSetAttribute(k_decode_int8_sm100<16, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(k_decode_int8_sm100<16, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kMaxSmemOptin) != cudaSuccess ||
             cudaFuncSetAttribute(k_gemm_int8_2sm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kG2SmemBytes) != cudaSuccess ||
@@ -241,7 +241,7 @@ uint32_t fp16_threshold_bits2(float thr) {
 // one K range of the cluster's `tiles` 128-channel tiles), a TMA ring of
 // `stages` 16 KB boxes, and the shared-memory offsets.
 struct DecodePlan {
-    int cluster, tiles, stages, groups, grid, mr;  // mr: rows of X per thread (8 or 16)
+    int cluster, tiles, stages, groups, grid, mr;  // mr: rows per chunk group (8 or 16)
     uint32_t off_xq, off_mask, off_pre, off_list, off_xo, off_oslot, off_red, off_bars, bytes;
 };
 
@@ -250,11 +250,11 @@ struct DecodePlan {
 bool decode_plan(int M, int K, int N, int cap, int sms, DecodePlan* P) {
     if (M < 1 || M > kMaxDecodeRows) return false;
     const int kbt = cdiv(K, 128);
-    const int rc = M <= 8 ? 2 : 1;  // 8-column chunks per X-side thread
+    // a CTA's K range holds at most kDecPro 8-column chunks (kP * kDecPro / kR)
     int cl = 0;
     for (int c : {4, 8}) {
         const int cc = std::min(c, kbt);
-        if (cdiv(kbt, cc) * 16 <= rc * kDecPro) {
+        if (cdiv(kbt, cc) * 16 <= kDecPro) {
             cl = cc;
             break;
         }
@@ -277,7 +277,7 @@ bool decode_plan(int M, int K, int N, int cap, int sms, DecodePlan* P) {
     const size_t list = align_up((size_t)std::min(K, std::max(cap, 1)) * 2, 16);
     const size_t xo = (size_t)kDecSmemOutliers * 16 * 2;
     const size_t oslot = (size_t)kDecSmemOutliers * 4;
-    const size_t red = (size_t)16 * kDecTileN * 4;
+    const size_t red = (size_t)cl * kDecTileN * 8 * groups * 4;  // one partial-sum slot per CTA of the cluster
     const size_t fixed = xq + mask + pre + list + xo + oslot + red;
     for (int s = 16; s >= 4; --s) {
         const size_t bars = (size_t)(2 * s + 5) * 8 + 256;
@@ -347,8 +347,8 @@ DecodeParams decode_params(const uint16_t* X, int M, const int8mm_weight* w, flo
 cudaError_t launch_decode(const DecodePlan& dp, const CUtensorMap& tm_w, const DecodeParams& p, cudaStream_t s,
                           bool pdl) {
     if (dp.mr == 8)
-        return launch_ex(k_decode_int8_sm100<8, 2>, dim3(dp.grid), dim3(kDecThreads), dp.bytes, s, pdl, dp.cluster, tm_w, p);
-    return launch_ex(k_decode_int8_sm100<16, 1>, dim3(dp.grid), dim3(kDecThreads), dp.bytes, s, pdl, dp.cluster, tm_w, p);
+        return launch_ex(k_decode_int8_sm100<8, 8>, dim3(dp.grid), dim3(kDecThreads), dp.bytes, s, pdl, dp.cluster, tm_w, p);
+    return launch_ex(k_decode_int8_sm100<16, 16>, dim3(dp.grid), dim3(kDecThreads), dp.bytes, s, pdl, dp.cluster, tm_w, p);
 }
 
 // ------------------------------------------------------------------ no-allocation decode forward

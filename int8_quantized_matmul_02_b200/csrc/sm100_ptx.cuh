@@ -197,9 +197,29 @@ __device__ __forceinline__ void atom_max_cluster_u32(uint32_t addr, uint32_t v) 
     asm volatile("atom.shared::cluster.max.u32 _, [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-// Relaxed atomic add (no return) on a 32-bit word of any CTA of the cluster.
-__device__ __forceinline__ void red_add_cluster_u32(uint32_t addr, uint32_t v) {
-    asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+// Asynchronous writes into the shared memory of any CTA of the cluster that
+// complete on an mbarrier of that CTA (transaction bytes = the size written):
+// the receiver's wait on the barrier makes them visible; the writer needs no
+// fence.  addr and mbar are shared::cluster addresses in the same CTA.
+__device__ __forceinline__ void st_async_u32(uint32_t addr, uint32_t v, uint32_t mbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];" ::"r"(addr), "r"(v),
+                 "r"(mbar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_async_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                            uint32_t mbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.u32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     addr),
+                 "r"(a), "r"(b), "r"(c), "r"(d), "r"(mbar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void red_async_max_u32(uint32_t addr, uint32_t v, uint32_t mbar) {
+    asm volatile(
+        "red.async.relaxed.cluster.shared::cluster.mbarrier::complete_tx::bytes.max.u32 [%0], %1, [%2];" ::"r"(addr),
+        "r"(v), "r"(mbar)
+        : "memory");
 }
 
 // Arrive (release at cluster scope) on an mbarrier of any CTA of the cluster.
@@ -225,6 +245,16 @@ __device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.ac
 // visible to the async proxy (tensor-core operand reads in any CTA).
 __device__ __forceinline__ void fence_proxy_async_cluster() {
     asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
+
+// The two halves of the whole-cluster barrier, for threads that have work to
+// do between arriving and waiting (every thread arrives once, then waits once).
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // Whole-cluster barrier: every thread of every CTA of the cluster.
