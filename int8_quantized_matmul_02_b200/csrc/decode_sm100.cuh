@@ -113,36 +113,50 @@ __device__ __forceinline__ uint2 dec_quant8(uint4 v, uint32_t fl, float scale) {
     return make_uint2(lo, hi);
 }
 
-// Max |x| (fp16 bits) over the columns of an 8-column chunk whose flag in fl
-// is clear: lanes of flagged columns are masked out, then a SIMD max tree.
-__device__ __forceinline__ uint32_t inlier_absmax_simd(uint4 v, uint32_t fl) {
-    uint32_t a0 = abs_bits2(v.x), a1 = abs_bits2(v.y), a2 = abs_bits2(v.z), a3 = abs_bits2(v.w);
-    if (fl) {
-        const uint32_t m0 = ((fl & 1u) ? 0u : 0xFFFFu) | ((fl & 2u) ? 0u : 0xFFFF0000u);
-        const uint32_t m1 = ((fl & 4u) ? 0u : 0xFFFFu) | ((fl & 8u) ? 0u : 0xFFFF0000u);
-        const uint32_t m2 = ((fl & 16u) ? 0u : 0xFFFFu) | ((fl & 32u) ? 0u : 0xFFFF0000u);
-        const uint32_t m3 = ((fl & 64u) ? 0u : 0xFFFFu) | ((fl & 128u) ? 0u : 0xFFFF0000u);
-        a0 &= m0;
-        a1 &= m1;
-        a2 &= m2;
-        a3 &= m3;
-    }
-    const uint32_t m = __vmaxu2(__vmaxu2(a0, a1), __vmaxu2(a2, a3));
-    return max(m & 0xFFFFu, m >> 16);
+// Pass (a) works on packed fp16 pairs with the native half2 compare and max:
+// |x| is the bit pattern with the sign cleared, __hge2_mask gives false for
+// NaN (so NaN is never an outlier) and __hmax2 returns the other operand when
+// one is NaN (so NaN never enters a row maximum).  thr2 holds, in both
+// halves, the smallest fp16 value >= the threshold (a NaN pattern when none
+// is, so nothing is flagged), so |x| >= thr  <=>  __hge2(|x|, thr2).
+__device__ __forceinline__ __half2 as_h2(uint32_t b) {
+    __half2 h;
+    memcpy(&h, &b, 4);
+    return h;
 }
 
-// Column flags (8 bits) of one chunk from its rows' |x| maxima (fp16 bits,
-// NaN already mapped to 0).  thr_bits2 holds, in both 16-bit lanes, the bits of
-// the smallest fp16 value >= the threshold (0x7C01 when no finite value and not
-// +inf reaches it), so |x| >= thr  <=>  bits(|x|) >= thr_bits as integers.
-__device__ __forceinline__ uint32_t chunk_flags(const uint32_t (&mx)[4], uint32_t thr_bits2) {
-    uint32_t fl = 0;
+__device__ __forceinline__ uint32_t as_u32(__half2 h) {
+    uint32_t b;
+    memcpy(&b, &h, 4);
+    return b;
+}
+
+__device__ __forceinline__ uint4 abs8(uint4 v) {
+    return make_uint4(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu, v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu);
+}
+
+// Outlier flags (bit j = column j) of one row's 8 columns from their |x|.
+__device__ __forceinline__ uint32_t flags8(uint4 a, __half2 thr2) {
+    const uint32_t m0 = __hge2_mask(as_h2(a.x), thr2), m1 = __hge2_mask(as_h2(a.y), thr2);
+    const uint32_t m2 = __hge2_mask(as_h2(a.z), thr2), m3 = __hge2_mask(as_h2(a.w), thr2);
+    return (m0 & 1u) | ((m0 >> 15) & 2u) | ((m1 & 1u) << 2) | ((m1 >> 13) & 8u) | ((m2 & 1u) << 4) |
+           ((m2 >> 11) & 32u) | ((m3 & 1u) << 6) | ((m3 >> 9) & 128u);
+}
+
+// Per-lane max of |x| over the columns whose flag in fl is clear (flagged
+// lanes count as +0).
+__device__ __forceinline__ __half2 inlier_max8(uint4 a, uint32_t fl) {
+    if (fl) {
+        uint32_t k[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t ge = __vcmpgeu2(mx[i], thr_bits2);  // 0xFFFF per lane where mx >= thr
-        fl |= ((ge & 1u) << (2 * i)) | (((ge >> 16) & 1u) << (2 * i + 1));
+        for (int w = 0; w < 4; ++w)
+            k[w] = (((fl >> (2 * w)) & 1u) ? 0u : 0xFFFFu) | (((fl >> (2 * w + 1)) & 1u) ? 0u : 0xFFFF0000u);
+        a.x &= k[0];
+        a.y &= k[1];
+        a.z &= k[2];
+        a.w &= k[3];
     }
-    return fl;
+    return __hmax2(__hmax2(as_h2(a.x), as_h2(a.y)), __hmax2(as_h2(a.z), as_h2(a.w)));
 }
 
 // kR: rows per 8-column chunk group (8 or 16, >= M); kP: (chunk, row) pairs
@@ -189,52 +203,61 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const int cid = blockIdx.x / CL;
     const int tile0 = cid * p.tiles_per_cluster;
     const int nt = max(0, min(p.tiles_per_cluster, p.num_tiles - tile0));
-    const int kb_lo = (int)((long long)p.kb_total * rank / CL);
-    const int kb_hi = (int)((long long)p.kb_total * (rank + 1) / CL);
+    const int kb_lo = p.kb_total * rank / CL;  // kb_total <= 1024, CL <= 8: no overflow
+    const int kb_hi = p.kb_total * (rank + 1) / CL;
     const int c0 = kb_lo * 16, c1 = min(nchunk, kb_hi * 16);
     const bool owner = rank < nt;
     const bool has_acc = nt > 0 && kb_hi > kb_lo;
     const uint32_t tmem_cols = p.tiles_per_cluster <= 1 ? 32u : (p.tiles_per_cluster <= 2 ? 64u : (p.tiles_per_cluster <= 4 ? 128u : 256u));
 
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < p.stages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+    // Set-up is split by role so that the X-side steps, which gate the first
+    // MMA, start at once: warp 0 initialises the mbarriers and starts the
+    // weight stream, warp 1 allocates TMEM, the X-side warps clear their
+    // buffers and load X.  Named barrier 2 ("mbarriers initialised, TMEM
+    // allocated"): warp 0 arrives, everyone else waits on it before the
+    // first use.  Peers write into this CTA only after the cluster barrier
+    // completes; every thread arrives once its part of the set-up is done and
+    // waits just before its first access to a peer (the weight stream needs
+    // no peer).
+    uint32_t tmem_base = 0;
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int s = 0; s < p.stages; ++s) {
+                mbar_init(&full[s], 1);
+                mbar_init(&empty[s], 1);
+            }
+            mbar_init(tfull, 1);
+            mbar_init(xq_ready, 1);
+            mbar_init(drain, 1);
+            mbar_init(xchg, 1);
+            mbar_init(red_done, 1);
+            *abort_flag = 0;
+            fence_mbar_init();
+            prefetch_tmap(&tm_w);
+            // bytes the peers will store: their flag words and M row maxima
+            // each, and (owner) one partial-sum slot per CTA of the cluster
+            uint32_t xb = 0;
+            for (int q = 0; q < CL; ++q) {
+                if (q == rank) continue;
+                const int qlo = p.kb_total * q / CL, qhi = p.kb_total * (q + 1) / CL;
+                xb += (uint32_t)(((min(nchunk, qhi * 16) + 3) / 4 - qlo * 4) * 4 + M * 4);
+            }
+            if (xb) mbar_arrive_expect_tx(xchg, xb);
+            else mbar_arrive(xchg);
+            if (owner && has_acc) mbar_arrive_expect_tx(red_done, (uint32_t)(CL * kDecTileN * RS * 4));
         }
-        mbar_init(tfull, 1);
-        mbar_init(xq_ready, 1);
-        mbar_init(drain, 1);
-        mbar_init(xchg, 1);
-        mbar_init(red_done, 1);
-        *abort_flag = 0;
-        fence_mbar_init();
-        prefetch_tmap(&tm_w);
-        // bytes the peers will store: their flag words and M row maxima each,
-        // and (owner) one partial-sum slot per CTA of the cluster
-        uint32_t xb = 0;
-        for (int q = 0; q < CL; ++q) {
-            if (q == rank) continue;
-            const int qlo = (int)((long long)p.kb_total * q / CL), qhi = (int)((long long)p.kb_total * (q + 1) / CL);
-            xb += (uint32_t)(((min(nchunk, qhi * 16) + 3) / 4 - qlo * 4) * 4 + M * 4);
-        }
-        if (xb) mbar_arrive_expect_tx(xchg, xb);
-        else mbar_arrive(xchg);
-        if (owner && has_acc) mbar_arrive_expect_tx(red_done, (uint32_t)(CL * kDecTileN * RS * 4));
-    }
-    if (warp == 1) {
+        __syncwarp();
+        cluster_arrive();
+        named_bar_arrive(2, kDecThreads);
+    } else if (warp == 1) {
         tmem_alloc(tmem_slot, tmem_cols);
         tmem_relinquish();
+        tc_fence_before();
+        cluster_arrive();
+        named_bar_sync(2, kDecThreads);
+        tc_fence_after();
+        tmem_base = *tmem_slot;
     }
-    if (threadIdx.x < 16) sra_bits[threadIdx.x] = 0u;
-    for (int w = threadIdx.x; w < nw; w += kDecThreads) smask[w] = 0u;
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    // Peers write into this CTA's barriers and buffers only after the cluster
-    // barrier completes; each thread arrives here and waits just before its
-    // first access to a peer (the weight stream needs no peer).
-    cluster_arrive();
-    const uint32_t tmem_base = *tmem_slot;
     pdl_launch_dependents();
 
     if (warp == 0) {
@@ -311,7 +334,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     } else {
         // ------------------------------------------------ X-side steps (warps 2..11)
         const int pt = threadIdx.x - 64;  // 0 .. kDecPro-1
-        pdl_wait();                       // X belongs to earlier work on the stream
+        if (pt < 16) sra_bits[pt] = 0u;
+        for (int w = pt; w < nw; w += kDecPro) smask[w] = 0u;
+        named_bar_sync(1, kDecPro);
+        cluster_arrive();
+        pdl_wait();  // X belongs to earlier work on the stream
         // (a) Thread pairs (8-column chunk, row): the kR rows of a chunk sit in
         // kR consecutive lanes, so a chunk's outlier flags are the OR of its
         // lanes' flags (shuffles), and a thread's row is the same for all its
@@ -319,36 +346,51 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         // and one scale per thread.  The values stay in registers for (b).
         const int prow = lane % kR;
         const bool row_ok = prow < M;
+        // iterations that hold any pair of this CTA (the same for every thread)
+        const int nit = ((c1 - c0) * kR + kDecPro - 1) / kDecPro;
         uint4 xv[kP];
         uint32_t cfl[kP];
 #pragma unroll
         for (int i = 0; i < kP; ++i) {
             const int c = c0 + (pt + i * kDecPro) / kR;
-            if (row_ok && c < c1) xv[i] = __ldg(reinterpret_cast<const uint4*>(Xg + (size_t)prow * K) + c);
+            if (i < nit && row_ok && c < c1) xv[i] = __ldg(reinterpret_cast<const uint4*>(Xg + (size_t)prow * K) + c);
         }
         {
-            uint32_t rmax = 0;
+            // in phases over the iterations, so that their dependency chains
+            // (compare, shuffles, mask, max) overlap
+            const __half2 thr2 = as_h2(p.thr_bits2);
+            __half2 rmax2 = as_h2(0u);
 #pragma unroll
             for (int i = 0; i < kP; ++i) {
                 const int c = c0 + (pt + i * kDecPro) / kR;
-                const bool ok = row_ok && c < c1;
-                uint32_t fl = 0;
-                if (ok) {
-                    const uint32_t mx[4] = {abs_bits2(xv[i].x), abs_bits2(xv[i].y), abs_bits2(xv[i].z),
-                                            abs_bits2(xv[i].w)};
-                    fl = chunk_flags(mx, p.thr_bits2);
-                }
-#pragma unroll
-                for (int off = 1; off < kR; off <<= 1) fl |= __shfl_xor_sync(0xffffffffu, fl, off);
-                cfl[i] = fl;
-                if (prow == 0 && c < c1 && fl) atomicOr(&smask[c >> 2], fl << ((c & 3) * 8));
-                if (ok) rmax = max(rmax, inlier_absmax_simd(xv[i], fl));
+                cfl[i] = (i < nit && row_ok && c < c1) ? flags8(abs8(xv[i]), thr2) : 0u;
             }
+#pragma unroll
+            for (int off = 1; off < kR; off <<= 1) {
+#pragma unroll
+                for (int i = 0; i < kP; ++i)
+                    if (i < nit) cfl[i] |= __shfl_xor_sync(0xffffffffu, cfl[i], off);
+            }
+#pragma unroll
+            for (int i = 0; i < kP; ++i) {
+                const int c = c0 + (pt + i * kDecPro) / kR;
+                if (i < nit && c < c1) {
+                    if (prow == 0 && cfl[i]) atomicOr(&smask[c >> 2], cfl[i] << ((c & 3) * 8));
+                    if (row_ok) rmax2 = __hmax2(rmax2, inlier_max8(abs8(xv[i]), cfl[i]));
+                }
+            }
+            // non-negative fp16 bit patterns order like their values
+            const uint32_t rb = as_u32(rmax2);
+            uint32_t rmax = max(rb & 0xFFFFu, rb >> 16);
 #pragma unroll
             for (int off = kR; off < 32; off <<= 1) rmax = max(rmax, __shfl_xor_sync(0xffffffffu, rmax, off));
             if (lane < kR && row_ok && rmax) atomicMax(&sra_bits[prow], rmax);
         }
-        named_bar_sync(1, kDecPro);
+        // every X-side thread's flags and maxima are in; the mbarriers are
+        // initialised and TMEM is allocated
+        named_bar_sync(2, kDecThreads);
+        tc_fence_after();
+        tmem_base = *tmem_slot;
         // this CTA's flag words (its K range covers whole words) and row
         // maxima to every peer; the peers' arrive the same way
         if (CL > 1) {
@@ -378,7 +420,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
             for (int i = 0; i < kP; ++i) {
                 const int c = c0 + (pt + i * kDecPro) / kR;
-                if (row_ok && c < c1) {
+                if (i < nit && row_ok && c < c1) {
                     const uint2 q = dec_quant8(xv[i], cfl[i], scl);
                     *reinterpret_cast<uint2*>(sxq + dec_xq_off(prow, (c - c0) * 8, p.groups)) = q;
                     if ((int)blockIdx.x < CL) *reinterpret_cast<uint2*>(p.xq_out + (size_t)prow * K + (size_t)c * 8) = q;
@@ -534,7 +576,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
 
     if (warp < 2) cluster_wait();  // the X-side warps waited before their first peer access
-    // after a timeout a peer's store may still be on its way here: let it land
+    // Every write into this CTA's shared memory (the peers' flag words, row
+    // maxima and partial sums) completes on a barrier this CTA has waited for,
+    // so it may leave without a closing cluster barrier; after a timeout a
+    // peer's store may still be on its way here: let it land first.
     if (*abort_flag) settle_after_abort();
     tc_fence_before();
     __syncthreads();
@@ -542,7 +587,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem_base, tmem_cols);
     }
-    cluster_sync_all();  // no CTA leaves while a peer may still write to it
 }
 
 }  // namespace i8mm
