@@ -269,7 +269,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             bool ok = true;
             for (int j = 0; ok && j < nt; ++j) {
                 for (int kb = kb_lo; kb < kb_hi; ++kb) {
-                    if (!wait_bounded(&empty[stage], phase ^ 1, wctx)) {
+                    if (!wait_bounded_sleep(&empty[stage], phase ^ 1, wctx)) {
                         ok = false;
                         break;
                     }
@@ -300,31 +300,30 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             const uint64_t db_step = (uint64_t)((p.groups * 1024) >> 4);
             int stage = 0;
             uint32_t phase = 0;
-            bool issued = false, ok = wait_bounded(xq_ready, 0, wctx);
+            bool issued = false, ok = wait_bounded_sleep(xq_ready, 0, wctx);
             tc_fence_after();
+            uint64_t da = da0;  // descriptor of the current ring stage
             for (int j = 0; ok && j < nt; ++j) {
                 const uint32_t dtm = tmem_base + (uint32_t)(32 * j);
                 uint64_t db = db0;
                 for (int kb = kb_lo; kb < kb_hi; ++kb) {
-                    if (!mbar_try_wait(&full[stage], phase) && !wait_bounded(&full[stage], phase, wctx)) {
+                    if (!mbar_try_wait(&full[stage], phase) && !wait_bounded_sleep(&full[stage], phase, wctx)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t da = da0 + (uint64_t)(stage * (kDecStageBytes >> 4));
-                    mma_s8(dtm, da, db, idesc, kb != kb_lo ? 1u : 0u);
-                    mma_s8(dtm, da + 2, db + 2, idesc, 1u);
-                    mma_s8(dtm, da + 4, db + 4, idesc, 1u);
-                    mma_s8(dtm, da + 6, db + 6, idesc, 1u);
+                    mma_s8_k128_commit(dtm, da, db, idesc, kb != kb_lo ? 1u : 0u, &empty[stage]);
                     db += db_step;
                     issued = true;
-                    tc_commit(&empty[stage]);
+                    da += (uint64_t)(kDecStageBytes >> 4);
                     if (++stage == p.stages) {
                         stage = 0;
                         phase ^= 1;
+                        da = da0;
                     }
                 }
             }
+
             if (ok) tc_commit(tfull);
             if (issued) {
                 tc_commit(drain);
@@ -410,7 +409,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         } else {
             cluster_wait();
         }
-        wait_bounded(xchg, 0, wctx);
+        wait_bounded_sleep(xchg, 0, wctx);
         // the whole mask and the row maxima are here: this thread's scale,
         // then (b) the int8 codes of its pairs into the shared B operand; the
         // first cluster also writes them to the workspace
@@ -529,7 +528,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             // partial sums of every tile of this CTA into this CTA's slot of the
             // tile owner's buffer (16-byte asynchronous stores, rows of one
             // channel together), completing on the owner's barrier
-            if (has_acc && __all_sync(0xffffffffu, wait_bounded(tfull, 0, wctx))) {
+            if (has_acc && __all_sync(0xffffffffu, wait_bounded_sleep(tfull, 0, wctx))) {
                 tc_fence_after();
                 for (int j = 0; j < nt; ++j) {
                     uint32_t r[16];
@@ -545,7 +544,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     }
                 }
             }
-            if (owner && has_acc && __all_sync(0xffffffffu, wait_bounded(red_done, 0, wctx)) && n < N) {
+            if (owner && has_acc && __all_sync(0xffffffffu, wait_bounded_sleep(red_done, 0, wctx)) && n < N) {
                 uint32_t sum[16];
 #pragma unroll
                 for (int m = 0; m < 16; ++m) sum[m] = 0u;

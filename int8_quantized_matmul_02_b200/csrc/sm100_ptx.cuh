@@ -84,6 +84,37 @@ __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const 
     }
 }
 
+// try_wait that may suspend the thread in hardware for up to hint_ns while the
+// phase is incomplete; it resumes when the phase completes, so a waiting warp
+// issues almost nothing (no hot polling that takes issue slots from the warps
+// doing the work).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// wait_bounded built on the suspending try_wait: the abort flag and the time
+// limit are checked each time the thread resumes (at least every 20 us).
+__device__ __noinline__ bool wait_bounded_sleep(uint64_t* bar, uint32_t parity, const WaitCtx& c) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (*c.abort_flag) return false;
+        if (globaltimer_ns() - t0 > c.limit_ns) {
+            raise_abort(c);
+            return false;
+        }
+    }
+}
+
 // wait_bounded with acquire at cluster scope (the barrier's arrivals come from
 // other CTAs of the cluster).
 __device__ __noinline__ bool wait_bounded_cluster(uint64_t* bar, uint32_t parity, const WaitCtx& c);
@@ -319,6 +350,29 @@ __device__ __forceinline__ void mma_s8(uint32_t d_tmem, uint64_t a_desc, uint64_
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}\n" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(z)
+        : "memory");
+}
+
+// One 128-byte K block of s8 MMAs (4 x K = 32, the K slices 32 bytes = +2 in
+// the descriptors' address field apart), then a commit of everything issued
+// so far to `bar`, as one asm block: a single thread issues every MMA, and for
+// small N its per-instruction overhead, not the tensor core, sets the rate.
+// The first MMA accumulates if `accumulate` is non-zero, the others always.
+__device__ __forceinline__ void mma_s8_k128_commit(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                   uint32_t accumulate, uint64_t* bar) {
+    const uint32_t z = 0, one = 1;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t.reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.ne.b32 q, %6, 0;\n\t"
+        "add.s64 a1, %1, 2;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 a3, %1, 6;\n\t"
+        "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], a1, b1, %3, {%5, %5, %5, %5}, q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], a2, b2, %3, {%5, %5, %5, %5}, q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], a3, b3, %3, {%5, %5, %5, %5}, q;\n\t"
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%7];\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(z), "r"(one), "r"(smem_u32(bar))
         : "memory");
 }
 
