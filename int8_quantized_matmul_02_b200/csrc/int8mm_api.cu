@@ -617,10 +617,10 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
         e = launch(k_detect, dim3(gx, gy), dim3(256), 0, s, false, X, M, K, threshold, rows, mask);
     }
     if (e == cudaSuccess) {
-        const int grid = std::max(1, std::min(cdiv(M, 8), sms * 4));
         const size_t smem = (size_t)cdiv(K, 32) * 8;
-        e = launch(k_quant_rows, dim3(grid), dim3(256), smem, s, true, X, M, K, (const uint32_t*)mask, max_outliers,
-                   kp, xq, ra, xo, idx, n_out, status);
+        const int grid = std::max(1, std::min(cdiv(M, 8), sms * 4));
+        e = launch(k_quant_rows, dim3(grid), dim3(256), smem, s, true, X, M, K, (const uint32_t*)mask,
+                   max_outliers, kp, xq, ra, xo, idx, n_out, status);
     }
     if (e == cudaSuccess)
         e = launch(k_gather_wo, dim3(cdiv(N, 64)), dim3(256), 0, s, true, (const int8_t*)w->wq,
@@ -635,7 +635,15 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
         p.num_m_blocks = cdiv(M, pair ? kG2BM : kGemmBM);
         p.num_n_blocks = cdiv(N, pair ? kG2BN : kGemmBN);
         p.num_tiles = p.num_m_blocks * p.num_n_blocks;
-        p.group_m = std::min(pair ? 8 : 16, p.num_m_blocks);
+        // Raster: a group of row blocks sweeps all column tiles before the next
+        // group starts; the group's band of Xq (group x tile rows x K bytes)
+        // stays in L2 while each W column tile is read once per group.  Use
+        // the largest group whose band fits in 48 MB (at least 8 row blocks).
+        {
+            const uint64_t band = (uint64_t)(pair ? kG2BM : kGemmBM) * (uint64_t)K;
+            const int fit = (int)std::min<uint64_t>(1u << 20, (48ull << 20) / band);
+            p.group_m = std::min(std::max(8, fit), p.num_m_blocks);
+        }
         p.kb_int8 = cdiv(K, 128);
         p.n_outliers = n_out;
         p.cap = max_outliers;

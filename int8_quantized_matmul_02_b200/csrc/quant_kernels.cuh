@@ -213,11 +213,24 @@ __device__ __forceinline__ uint2 quant8_plain(uint4 v, float scale) {
     return make_uint2(lo, hi);
 }
 
-// Max |x| (fp16 bits) of an 8-column chunk with no outlier column.
-__device__ __forceinline__ uint32_t chunk_absmax_plain(uint4 v) {
-    const uint32_t m = __vmaxu2(__vmaxu2(abs_bits2(v.x), abs_bits2(v.y)), __vmaxu2(abs_bits2(v.z), abs_bits2(v.w)));
-    return max(m & 0xFFFFu, m >> 16);
+// Max |x| (fp16 bits) of an 8-column chunk with no outlier column, on packed
+// fp16 pairs with the native half2 max: |x| is the bit pattern with the sign
+// cleared, and __hmax2 returns the other operand when one is NaN, so a NaN
+// never wins (a lane whose 8 values are all NaN gives the +0 of the start).
+__device__ __forceinline__ uint32_t chunk_absmax_h2(uint4 v) {
+    __half2 a0, a1, a2, a3;
+    const uint32_t b0 = v.x & 0x7FFF7FFFu, b1 = v.y & 0x7FFF7FFFu, b2 = v.z & 0x7FFF7FFFu, b3 = v.w & 0x7FFF7FFFu;
+    memcpy(&a0, &b0, 4);
+    memcpy(&a1, &b1, 4);
+    memcpy(&a2, &b2, 4);
+    memcpy(&a3, &b3, 4);
+    const __half2 zero = __floats2half2_rn(0.0f, 0.0f);
+    const __half2 m = __hmax2(zero, __hmax2(__hmax2(a0, a1), __hmax2(a2, a3)));
+    uint32_t mb;
+    memcpy(&mb, &m, 4);
+    return max(mb & 0xFFFFu, mb >> 16);
 }
+
 
 // Quantise one 8-column chunk c of a row; outlier columns give 0 and are
 // copied to their slot of the row's fp16 outlier vector.
@@ -327,7 +340,7 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
                 const int c = c0 + 32 * i;
                 if (c < nchunk) {
                     const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
-                    amax = max(amax, fl ? chunk_inlier_absmax(v[i], smask, c) : chunk_absmax_plain(v[i]));
+                    amax = max(amax, fl ? chunk_inlier_absmax(v[i], smask, c) : chunk_absmax_h2(v[i]));
                 }
             }
         }
