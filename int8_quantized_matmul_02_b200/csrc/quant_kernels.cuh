@@ -172,21 +172,6 @@ __device__ __forceinline__ uint32_t chunk_inlier_absmax(uint4 v, const uint32_t*
     return amax;
 }
 
-// Max |x| over the columns of one 8-column chunk whose outlier flag (bit j of
-// fl) is clear, as fp16 bits.
-__device__ __forceinline__ uint32_t inlier_absmax_flags(uint4 v, uint32_t fl) {
-    const uint32_t h[4] = {v.x, v.y, v.z, v.w};
-    uint32_t amax = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint32_t a = abs_bits2(h[j]);
-        const uint32_t lo = ((fl >> (2 * j)) & 1u) ? 0u : (a & 0xFFFFu);
-        const uint32_t hi = ((fl >> (2 * j + 1)) & 1u) ? 0u : (a >> 16);
-        amax = max(amax, max(lo, hi));
-    }
-    return amax;
-}
-
 // round_half_even(x * scale) clamped to [-127, 127], with the rounding done by
 // adding 1.5 * 2^23 in fp32: for |v| < 2^22 the sum RN(v + 1.5*2^23) keeps
 // round_half_even(v) in its low mantissa bits, so the result equals

@@ -166,14 +166,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
         : "memory");
 }
 
-// Contiguous copy of `bytes` (a multiple of 16, both addresses 16-byte
-// aligned) from global to shared memory; completes on `bar`.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_u32(dst)),
-                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-                 : "memory");
-}
 
 // 2-D tiled store of one box from shared memory (bulk-group completion).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int x, int y) {
@@ -216,18 +208,6 @@ __device__ __forceinline__ uint32_t map_to_rank(const void* local, uint32_t rank
     return r;
 }
 
-__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ void st_cluster_v2(uint32_t addr, uint2 v) {
-    asm volatile("st.shared::cluster.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(v.x), "r"(v.y) : "memory");
-}
-
-__device__ __forceinline__ void atom_max_cluster_u32(uint32_t addr, uint32_t v) {
-    asm volatile("atom.shared::cluster.max.u32 _, [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-
 // Asynchronous writes into the shared memory of any CTA of the cluster that
 // complete on an mbarrier of that CTA (transaction bytes = the size written):
 // the receiver's wait on the barrier makes them visible; the writer needs no
@@ -268,14 +248,6 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
         : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
-}
-
-__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
-
-// Make this thread's generic-proxy writes to shared memory of the cluster
-// visible to the async proxy (tensor-core operand reads in any CTA).
-__device__ __forceinline__ void fence_proxy_async_cluster() {
-    asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
 }
 
 // The two halves of the whole-cluster barrier, for threads that have work to
