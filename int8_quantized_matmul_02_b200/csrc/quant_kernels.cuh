@@ -172,32 +172,27 @@ __device__ __forceinline__ uint32_t chunk_inlier_absmax(uint4 v, const uint32_t*
     return amax;
 }
 
-// round_half_even(x * scale) clamped to [-127, 127], with the rounding done by
-// adding 1.5 * 2^23 in fp32: for |v| < 2^22 the sum RN(v + 1.5*2^23) keeps
-// round_half_even(v) in its low mantissa bits, so the result equals
-// __float2int_rn(v) exactly (here |v| <= 127.0001) at full fp32 rate.
-__device__ __forceinline__ int quant1_fast(float x, float scale) {
-    const float r = __fadd_rn(__fmul_rn(x, scale), 12582912.0f);
-    return max(-127, min(127, __float_as_int(r) - 0x4B400000));
-}
-
-// Codes of an 8-column chunk with no outlier column (the common case).
+// Codes of an 8-column chunk with no outlier column (the common case).  Every
+// value is a non-outlier of its row, so |x| <= ra and |x * scale| <= 127 * (1
+// + 2^-24): RN32(RN32(x * scale) + 1.5 * 2^23) holds the code in its low
+// byte (no clamp can trigger), and the bytes are packed straight from the
+// float bit patterns.  (A NaN in X, outside the method's inputs, gets an
+// unspecified code.)
 __device__ __forceinline__ uint2 quant8_plain(uint4 v, float scale) {
     const uint32_t h[4] = {v.x, v.y, v.z, v.w};
-    int q[8];
+    uint32_t b[8];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[j]));
-        q[2 * j] = quant1_fast(f.x, scale);
-        q[2 * j + 1] = quant1_fast(f.y, scale);
+        b[2 * j] = __float_as_uint(__fadd_rn(__fmul_rn(f.x, scale), 12582912.0f));
+        b[2 * j + 1] = __float_as_uint(__fadd_rn(__fmul_rn(f.y, scale), 12582912.0f));
     }
-    const uint32_t lo = __byte_perm(__byte_perm((uint32_t)q[0], (uint32_t)q[1], 0x0040),
-                                    __byte_perm((uint32_t)q[2], (uint32_t)q[3], 0x0040), 0x5410);
-    const uint32_t hi = __byte_perm(__byte_perm((uint32_t)q[4], (uint32_t)q[5], 0x0040),
-                                    __byte_perm((uint32_t)q[6], (uint32_t)q[7], 0x0040), 0x5410);
+    // __byte_perm(a, b, 0x0040) puts the low bytes of a and b in bytes 0 and
+    // 1; 0x5410 joins two such halves
+    const uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+    const uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
     return make_uint2(lo, hi);
 }
-
 // Max |x| (fp16 bits) of an 8-column chunk with no outlier column, on packed
 // fp16 pairs with the native half2 max: |x| is the bit pattern with the sign
 // cleared, and __hmax2 returns the other operand when one is NaN, so a NaN
