@@ -130,10 +130,13 @@ int8mm_status int8mm_forward(const uint16_t* X, int M, const int8mm_weight* w, f
                              void* stream);
 
 enum {
-    INT8MM_PATH_AUTO = 0,    /* decode kernel for M <= 16, tiled GEMM otherwise */
+    INT8MM_PATH_AUTO = 0,    /* decode kernel for M <= 16 when it fits (K <= 20480 and its
+                                shared-memory plan), tiled GEMM otherwise */
     INT8MM_PATH_GEMM = 1,    /* detect -> quantise -> gather -> tcgen05 GEMM, any M (SM-pair
                                 256 x 256 tiles when M > 128) */
-    INT8MM_PATH_DECODE = 2,  /* single fused weight-streaming kernel, M <= 16 */
+    INT8MM_PATH_DECODE = 2,  /* single fused weight-streaming kernel (clusters of CTAs split K),
+                                M <= 16, K <= 20480 and its shared-memory plan fits;
+                                INT8MM_ERR_INVALID_ARGUMENT otherwise */
     INT8MM_PATH_GEMM_1SM = 3 /* the tiled path with single-SM 128 x 256 GEMM tiles (for tests) */
 };
 

@@ -113,6 +113,11 @@ def test_forced_decode_path_needs_small_m(lib):
     assert _fwd(lib, M=17, opts=_abi.ForwardOpts(_abi.PATH_DECODE, None, 0)) == 1
 
 
+def test_forced_decode_path_needs_k_within_its_limit(lib):
+    # a cluster of 8 CTAs splits K; each CTA's range must fit its X-side threads (K <= 20480)
+    assert _fwd(lib, M=8, w=_weight(K=20608), opts=_abi.ForwardOpts(_abi.PATH_DECODE, None, 0)) == 1
+
+
 def test_prepare_rejects_bad_keep_lists(lib):
     out = _abi.Weight()
     keep = (ctypes.c_int32 * 3)(5, 3, 9)  # not ascending
