@@ -617,7 +617,8 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
         e = launch(k_detect, dim3(gx, gy), dim3(256), 0, s, false, X, M, K, threshold, rows, mask);
     }
     if (e == cudaSuccess) {
-        const size_t smem = (size_t)cdiv(K, 32) * 8;
+        // mask words, their prefix counts, and one flag word per 2048-column window
+        const size_t smem = ((size_t)cdiv(K, 32) * 2 + (size_t)cdiv(K, 2048)) * 4;
         const int grid = std::max(1, std::min(cdiv(M, 8), sms * 4));
         e = launch(k_quant_rows, dim3(grid), dim3(256), smem, s, true, X, M, K, (const uint32_t*)mask,
                    max_outliers, kp, xq, ra, xo, idx, n_out, status);

@@ -284,6 +284,17 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
         carry += blk_total;
         __syncthreads();
     }
+    // A warp's iteration covers 256 chunks (2048 columns, 64 mask words); a
+    // window with no outlier column (the common case) skips the per-chunk
+    // flag lookups.
+    const int nchunk = K / 8;
+    const int nwin = (nchunk + 255) / 256;
+    uint32_t* swin = qsm + 2 * nw;
+    for (int t = tid; t < nwin; t += 256) {
+        uint32_t o = 0u;
+        for (int w = t * 64; w < min(nw, t * 64 + 64); ++w) o |= smask[w];
+        swin[t] = o;
+    }
     if (tid == 0) total_sh = carry;
     __syncthreads();
     const int total = total_sh;
@@ -306,12 +317,18 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
         }
     }
 
-    const int nchunk = K / 8;
     for (int m = blockIdx.x * 8 + warp; m < M; m += gridDim.x * 8) {
         const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)m * K);
         uint32_t amax = 0;
-        for (int c0 = lane; c0 < nchunk; c0 += 32 * 8) {
+        for (int c0 = lane, it = 0; c0 < nchunk; c0 += 32 * 8, ++it) {
             uint4 v[8];
+            if (swin[it] == 0u && (it + 1) * 256 <= nchunk) {  // whole window, no outlier column
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] = __ldg(xr + c0 + 32 * i);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) amax = max(amax, chunk_absmax_h2(v[i]));
+                continue;
+            }
 #pragma unroll
             for (int i = 0; i < 8; ++i)
                 if (c0 + 32 * i < nchunk) v[i] = __ldg(xr + c0 + 32 * i);
@@ -330,8 +347,15 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
         if (lane == 0) ra[m] = rmax;
         uint2* qr = reinterpret_cast<uint2*>(Xq + (size_t)m * K);
         uint16_t* xo_row = Xo + (size_t)m * kp;
-        for (int c0 = lane; c0 < nchunk; c0 += 32 * 8) {
+        for (int c0 = lane, it = 0; c0 < nchunk; c0 += 32 * 8, ++it) {
             uint4 v[8];
+            if (swin[it] == 0u && (it + 1) * 256 <= nchunk) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] = __ldg(xr + c0 + 32 * i);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) qr[c0 + 32 * i] = quant8_plain(v[i], scale);
+                continue;
+            }
 #pragma unroll
             for (int i = 0; i < 8; ++i)
                 if (c0 + 32 * i < nchunk) v[i] = __ldg(xr + c0 + 32 * i);
