@@ -133,7 +133,7 @@ class ClockSampler:
 KERNEL_SOURCES = {
     "k_gemm_int8_2sm": ("gemm2sm_sm100.cuh", "gemm_sm100.cuh", "sm100_ptx.cuh"),
     "k_gemm_int8_sm100": ("gemm_sm100.cuh", "sm100_ptx.cuh"),
-    "k_decode_int8_sm100": ("decode_sm100.cuh", "quant_kernels.cuh", "sm100_ptx.cuh"),
+    "k_decode_int8_sm100": ("decode_sm100.cuh", "sm100_ptx.cuh"),
 }
 
 

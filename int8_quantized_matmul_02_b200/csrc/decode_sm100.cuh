@@ -34,7 +34,6 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
-#include "quant_kernels.cuh"
 #include "sm100_ptx.cuh"
 
 namespace i8mm {
@@ -68,6 +67,10 @@ constexpr int kDecSmemOutliers = 128;        // outlier columns whose x values a
 constexpr int kDecTileN = 128;
 constexpr int kDecStageBytes = kDecTileN * 128;  // 16 KB
 constexpr int kDecMaxCluster = 8;
+
+__device__ __forceinline__ float dec_half_to_float(uint32_t bits16) {
+    return __half2float(__ushort_as_half((unsigned short)bits16));
+}
 
 // Byte offset of Xq[m, k] inside the shared B operand (k relative to the
 // CTA's K range): K-block kb = k/128 holds `groups` 8-row atoms of 1024 bytes;
@@ -414,7 +417,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         // then (b) the int8 codes of its pairs into the shared B operand; the
         // first cluster also writes them to the workspace
         {
-            const float rmax = row_ok ? half_bits_to_float(sra_bits[prow]) : 0.0f;
+            const float rmax = row_ok ? dec_half_to_float(sra_bits[prow]) : 0.0f;
             const float scl = rmax > 0.0f ? __fdiv_rn(127.0f, rmax) : 0.0f;
 #pragma unroll
             for (int i = 0; i < kP; ++i) {
@@ -427,7 +430,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             }
         }
         if (warp == 3 && lane < 16) {
-            const float rmax = half_bits_to_float(sra_bits[lane]);
+            const float rmax = dec_half_to_float(sra_bits[lane]);
             srs[lane] = __fdiv_rn(rmax, 16129.0f);
             if (blockIdx.x == 0 && lane < M) p.ra_out[lane] = rmax;
         }
@@ -501,28 +504,28 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     const int slot = soslot[j];
                     float w;
                     if (slot >= 0) {
-                        w = half_bits_to_float(p.w_keep[(size_t)slot * N + n]);
+                        w = dec_half_to_float(p.w_keep[(size_t)slot * N + n]);
                     } else {
                         const float tq = __fmul_rn((float)p.wq[(size_t)n * K + slist[j]], cav);
                         w = __half2float(__float2half_rn(__fdiv_rn(tq, 127.0f)));
                     }
 #pragma unroll
                     for (int m = 0; m < 16; ++m)
-                        if (m < M) o[m] = fmaf(half_bits_to_float(sxo[j * 16 + m]), w, o[m]);
+                        if (m < M) o[m] = fmaf(dec_half_to_float(sxo[j * 16 + m]), w, o[m]);
                 }
                 for (int j = n_fast; j < n_eff; ++j) {
                     const int k = slist[j];
                     const int slot = p.keep_slot[k];
                     float w;
                     if (slot >= 0) {
-                        w = half_bits_to_float(p.w_keep[(size_t)slot * N + n]);
+                        w = dec_half_to_float(p.w_keep[(size_t)slot * N + n]);
                     } else {
                         const float tq = __fmul_rn((float)p.wq[(size_t)n * K + k], cav);
                         w = __half2float(__float2half_rn(__fdiv_rn(tq, 127.0f)));
                     }
 #pragma unroll
                     for (int m = 0; m < 16; ++m)
-                        if (m < M) o[m] = fmaf(half_bits_to_float(Xg[(size_t)m * K + k]), w, o[m]);
+                        if (m < M) o[m] = fmaf(dec_half_to_float(Xg[(size_t)m * K + k]), w, o[m]);
                 }
             }
             // partial sums of every tile of this CTA into this CTA's slot of the

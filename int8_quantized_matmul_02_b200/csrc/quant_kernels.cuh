@@ -119,16 +119,26 @@ __global__ void __launch_bounds__(256) k_detect(const uint16_t* __restrict__ X, 
     const int col0 = blockIdx.x * 256 + lane * 8;
     const int row0 = blockIdx.y * rows_per_block;
     const int row1 = min(M, row0 + rows_per_block);
-    uint32_t m[4] = {0, 0, 0, 0};
+    // running |x| maxima as packed fp16 pairs: __hmax2 returns the other operand
+    // when one is NaN, so from the +0 start a NaN never enters a maximum
+    __half2 h[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(0.0f, 0.0f);
     if (col0 < K) {
         for (int r = row0 + warp; r < row1; r += 8) {
-            uint4 v = __ldg(reinterpret_cast<const uint4*>(X + (size_t)r * K + col0));
-            m[0] = __vmaxu2(m[0], abs_bits2(v.x));
-            m[1] = __vmaxu2(m[1], abs_bits2(v.y));
-            m[2] = __vmaxu2(m[2], abs_bits2(v.z));
-            m[3] = __vmaxu2(m[3], abs_bits2(v.w));
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(X + (size_t)r * K + col0));
+            const uint32_t a[4] = {v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu, v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                __half2 t;
+                memcpy(&t, &a[i], 4);
+                h[i] = __hmax2(h[i], t);
+            }
         }
     }
+    uint32_t m[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) memcpy(&m[i], &h[i], 4);
 #pragma unroll
     for (int i = 0; i < 4; ++i) red[warp][lane][i] = m[i];
     __syncthreads();
