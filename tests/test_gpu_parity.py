@@ -95,6 +95,9 @@ def test_gemm_path_zero_rows_and_columns():
     (9, 1024, 528, 3),
     (16, 4112, 400, 5),       # K not a multiple of 128, N not a multiple of 128
     (3, 2048, 11008, 1),
+    (4, 16, 272, 1),          # one 16-column K block: a cluster of one CTA
+    (5, 128, 1040, 2),        # one full K block
+    (16, 20480, 272, 7),      # the longest K the decode kernel takes (clusters of 8)
 ])
 def test_decode_path_matches_oracle(M, K, N, n_seed):
     _run_case(M, K, N, n_seed, path="decode", seed=M * 31 + K)
