@@ -7,7 +7,8 @@
 // ring from the moment the CTA starts and keeps the X-side steps that gate
 // the first tensor-core instruction short:
 //
-// Clusters of CL CTAs (CL = 4 or 8) split K: CTA r of a cluster owns the
+// Clusters of CL CTAs (4, or 8 for long K; as many as K has 128-column blocks
+// when that is fewer) split K: CTA r of a cluster owns the
 // r-th K range of the cluster's T (<= CL) 128-channel weight tiles.  It reads
 // only its K range of X, so the outlier flags of those columns are final at
 // once (all M rows of a column are in the same CTA), quantises only those
