@@ -28,6 +28,21 @@ MUTATIONS = {
     "wrong_denominator": ("v = v / 16129.0f;", "v = v / 16384.0f;"),
     "kept_row_ignored": ("if (slot >= 0) {\n                w = W_keep", "if (slot >= 1000000) {\n                w = W_keep"),
     "xo_wrong_column": ("Xo[(size_t)m * n_o + j] = row[idx[j]];", "Xo[(size_t)m * n_o + j] = row[idx[j] > 0 ? idx[j] - 1 : 0];"),
+    "threshold_signed": ("if (fabsf(x) >= thr)", "if (x >= thr)"),
+    "detect_first_row_only": ("for (int m = 0; m < M; ++m) {\n            float x = orc_half_to_float(X[",
+                              "for (int m = 0; m < 1; ++m) {\n            float x = orc_half_to_float(X["),
+    "outlier_list_descending": ("for (int k = 0; k < K; ++k) {\n        int flag = 0;",
+                                "for (int k = K - 1; k >= 0; --k) {\n        int flag = 0;"),
+    "row_absmax_signed": ("float a = fabsf(orc_half_to_float(row[k]));", "float a = orc_half_to_float(row[k]);"),
+    "weight_absmax_signed": ("float a = fabsf(orc_half_to_float(W[(size_t)k * N + n]));",
+                             "float a = orc_half_to_float(W[(size_t)k * N + n]);"),
+    "product_in_double": ("float r = nearbyintf(x * scale);", "float r = (float)nearbyint((double)x * (double)scale);"),
+    "epilogue_ra_twice": ("v = v * ca;", "v = v * ra;"),
+    "dequantised_row_over_128": ("w = orc_float_to_half(t / 127.0f);", "w = orc_float_to_half(t / 128.0f);"),
+    "outlier_weight_rows_reversed": ("orc_half_to_float(Wo[(size_t)j * N + n]);",
+                                     "orc_half_to_float(Wo[(size_t)(n_o - 1 - j) * N + n]);"),
+    "half_subnormal_exponent": ("v = ldexpf((float)mant, -24);", "v = ldexpf((float)mant, -25);"),
+    "half_encode_truncates": ("float m = nearbyintf(ldexpf(a, 10 - e));", "float m = truncf(ldexpf(a, 10 - e));"),
 }
 
 
@@ -35,6 +50,8 @@ def _pin_suite():
     """Run a fast subset of the pins; return the names of those that fail."""
     failed = []
     checks = {
+        "half_decode": pins.test_half_to_float_exhaustive,
+        "half_encode": pins.test_float_to_half_round_half_even,
         "worked_example": pins.test_worked_example_golden,
         "threshold_equality": pins.test_value_exactly_at_threshold_is_outlier,
         "absmax_127": pins.test_absmax_maps_to_127,
