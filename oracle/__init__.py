@@ -19,7 +19,12 @@ raw 16-bit patterns.  Each wrapper names the passage it follows:
   decomposition ... isolates the outlier feature dimensions into a 16-bit
   matrix multiplication");
 * weight conversion once at load -- the same abstract ("loaded, converted to
-  Int8, and used immediately").
+  Int8, and used immediately");
+* block-wise 8-bit codec -- the axolotl page's "8-Bit Optimizers" paragraphs
+  (blocks normalised by their own maximum, an 8-bit index per value);
+* group-wise matmul -- the scite report for nuQmm (nuQmm / ZeroQuant use one
+  constant per group, finer than vector-wise; GPTQ's grouping of consecutive
+  weights).
 """
 from __future__ import annotations
 
@@ -77,6 +82,19 @@ def _setup(lib):
     lib.orc_epilogue.restype = None
     lib.orc_forward_points.argtypes = [P, P, P, P, P, P, I, I, I, P, P, I, P, P]
     lib.orc_forward_points.restype = I
+    L = ctypes.c_long
+    lib.orc_block_quantize.argtypes = [P, L, I, P, P]
+    lib.orc_block_quantize.restype = None
+    lib.orc_block_dequantize.argtypes = [P, P, L, I, P]
+    lib.orc_block_dequantize.restype = None
+    lib.orc_quantize_rows_grouped.argtypes = [P, I, I, I, P, I, P, P, P]
+    lib.orc_quantize_rows_grouped.restype = None
+    lib.orc_quantize_weight_grouped.argtypes = [P, I, I, I, P, P]
+    lib.orc_quantize_weight_grouped.restype = None
+    lib.orc_gather_w_outlier_grouped.argtypes = [P, P, I, P, P, I, I, I, P, I, P]
+    lib.orc_gather_w_outlier_grouped.restype = None
+    lib.orc_grouped_forward.argtypes = [P, P, P, P, P, I, I, I, I, P, P]
+    lib.orc_grouped_forward.restype = I
     return lib
 
 
@@ -272,3 +290,110 @@ def forward_steps_abc(X: np.ndarray, prep: dict, threshold: float) -> dict:
     Wo = gather_w_outlier(prep, idx)
     return {"idx": idx, "xq": Xq, "ra": ra, "xo": Xo, "wo": Wo}
 
+
+
+# --------------------------------------------------------------------------
+# block-wise 8-bit codec
+# --------------------------------------------------------------------------
+
+def block_quantize(x: np.ndarray, B: int):
+    """fp32 vector -> (codes int8 n, absmax float32 ceil(n/B)); block b covers
+    [b*B, min(n, (b+1)*B)), each normalised by its own maximum."""
+    x = _c(np.ravel(x), np.float32)
+    n = int(x.size)
+    assert B >= 1
+    q = np.zeros(n, dtype=np.int8)
+    amax = np.zeros((n + B - 1) // B, dtype=np.float32)
+    _load().orc_block_quantize(_ptr(x), n, int(B), _ptr(q), _ptr(amax))
+    return q, amax
+
+
+def block_dequantize(q: np.ndarray, absmax: np.ndarray, B: int) -> np.ndarray:
+    """x' = (q * absmax[block]) / 127 in fp32."""
+    q = _c(np.ravel(q), np.int8)
+    absmax = _c(absmax, np.float32)
+    n = int(q.size)
+    assert absmax.size == (n + B - 1) // B
+    out = np.zeros(n, dtype=np.float32)
+    _load().orc_block_dequantize(_ptr(q), _ptr(absmax), n, int(B), _ptr(out))
+    return out
+
+
+# --------------------------------------------------------------------------
+# group-wise matmul (one constant per G consecutive inner-product indices)
+# --------------------------------------------------------------------------
+
+def quantize_rows_grouped(X: np.ndarray, idx: np.ndarray, G: int):
+    """-> (Xq int8 MxK, ra float32 M x K/G, Xo float16 M x n_o)."""
+    xb = _bits(X)
+    M, K = xb.shape
+    assert G >= 1 and K % G == 0
+    idx = _c(idx, np.int32)
+    Xq = np.zeros((M, K), dtype=np.int8)
+    ra = np.zeros((M, K // G), dtype=np.float32)
+    Xo = np.zeros((M, idx.size), dtype=np.uint16)
+    _load().orc_quantize_rows_grouped(_ptr(xb), M, K, int(G), _ptr(idx), idx.size, _ptr(Xq), _ptr(ra), _ptr(Xo))
+    return Xq, ra, Xo.view(np.float16)
+
+
+def quantize_weight_grouped(W: np.ndarray, G: int):
+    """W (K x N fp16) -> (Wq int8 N x K, ca float32 N x K/G)."""
+    wb = _bits(W)
+    K, N = wb.shape
+    assert G >= 1 and K % G == 0
+    Wq = np.zeros((N, K), dtype=np.int8)
+    ca = np.zeros((N, K // G), dtype=np.float32)
+    _load().orc_quantize_weight_grouped(_ptr(wb), K, N, int(G), _ptr(Wq), _ptr(ca))
+    return Wq, ca
+
+
+def prepare_weight_grouped(W: np.ndarray, keep_idx, G: int) -> dict:
+    Wq, ca = quantize_weight_grouped(W, G)
+    keep = np.asarray(sorted(set(int(k) for k in np.asarray(keep_idx).ravel())), dtype=np.int32)
+    w_keep = np.ascontiguousarray(np.asarray(W, dtype=np.float16)[keep, :])
+    return {"K": W.shape[0], "N": W.shape[1], "G": int(G), "wq": Wq, "ca": ca, "keep_idx": keep, "w_keep": w_keep}
+
+
+def gather_w_outlier_grouped(prep: dict, idx: np.ndarray) -> np.ndarray:
+    idx = _c(idx, np.int32)
+    keep = _c(prep["keep_idx"], np.int32)
+    wk = _bits(prep["w_keep"]) if keep.size else np.zeros((0, prep["N"]), dtype=np.uint16)
+    Wo = np.zeros((idx.size, prep["N"]), dtype=np.uint16)
+    _load().orc_gather_w_outlier_grouped(_ptr(wk), _ptr(keep), keep.size, _ptr(_c(prep["wq"], np.int8)),
+                                         _ptr(_c(prep["ca"], np.float32)), prep["K"], prep["N"], prep["G"],
+                                         _ptr(idx), idx.size, _ptr(Wo))
+    return Wo.view(np.float16)
+
+
+def grouped_product(Xq, ra, Wq, ca, G: int, o=None):
+    """-> (acc int32 M x N x K/G, Y float16 M x N)."""
+    Xq = _c(Xq, np.int8)
+    Wq = _c(Wq, np.int8)
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    assert Wq.shape[1] == K and K % G == 0
+    ng = K // G
+    ra = _c(ra, np.float32)
+    ca = _c(ca, np.float32)
+    assert ra.shape == (M, ng) and ca.shape == (N, ng)
+    op = ctypes.c_void_p(0)
+    if o is not None:
+        o = _c(o, np.float32)
+        op = _ptr(o)
+    acc = np.zeros((M, N, ng), dtype=np.int32)
+    Y = np.zeros((M, N), dtype=np.uint16)
+    rc = _load().orc_grouped_forward(_ptr(Xq), _ptr(ra), _ptr(Wq), _ptr(ca), op, M, N, K, int(G), _ptr(acc), _ptr(Y))
+    if rc != 0:
+        raise OverflowError("a group sum does not fit int32")
+    return acc, Y.view(np.float16)
+
+
+def forward_grouped(X: np.ndarray, prep: dict, threshold: float) -> dict:
+    """The group-wise forward pass; returns every intermediate and Y."""
+    G = prep["G"]
+    idx = detect_outliers(X, threshold)
+    Xq, ra, Xo = quantize_rows_grouped(X, idx, G)
+    Wo = gather_w_outlier_grouped(prep, idx)
+    o = outlier_gemm(Xo, Wo)
+    acc, Y = grouped_product(Xq, ra, prep["wq"], prep["ca"], G, o)
+    return {"idx": idx, "xq": Xq, "ra": ra, "xo": Xo, "acc": acc, "wo": Wo, "o": o, "y": Y}

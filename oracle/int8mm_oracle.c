@@ -35,6 +35,11 @@
  *     else from the dequantised int8 row fp16(q * ca / 127);
  *   - y = fp16( (float)acc * ra[m] * ca[n] / 16129 + o ), left to right.
  *
+ * Two variants follow the vector-wise matmul at the end of the file, with
+ * the same per-value rule: a block-wise linear 8-bit codec of an fp32 vector
+ * and the group-wise matmul (one constant per group of G consecutive inner
+ * indices).  The GPU library does not implement them yet.
+ *
  * Build: gcc -O2 -ffp-contract=off (no fast-math), -pthread.
  */
 #include <fenv.h>
@@ -336,4 +341,170 @@ int orc_forward_points(const int8_t* Xq, const float* ra, const int8_t* Wq, cons
         y_out[p] = combine(acc_out[p], ra[pm[p]], ca[pn[p]], o);
     }
     return rc;
+}
+
+/* ======================================================================== */
+/* Variants beyond the vector-wise matmul                                   */
+/* ======================================================================== */
+
+/* ------------------------------------------------------------------------ */
+/* Block-wise linear 8-bit codec of an fp32 vector.  The axolotl             */
+/* "llama3-model-quantization" summary ("8-Bit Optimizers") describes it for */
+/* optimizer state: cut the vector into blocks, normalise each block by its  */
+/* own maximum and store an 8-bit index per value, so an outlier coarsens    */
+/* only its own block.  Levels are linear (equal bins, "Key Points"); the    */
+/* rule per value is the matmul's: scale = 127/absmax, half-even rounding of */
+/* the fp32 product, clamp to [-127, 127]; absmax 0 gives codes 0.           */
+/* Block b covers [b*B, min(n, (b+1)*B)): the last block may be short.       */
+/* Inputs are finite.                                                        */
+/* ------------------------------------------------------------------------ */
+
+void orc_block_quantize(const float* x, long n, int B, int8_t* q, float* absmax) {
+    fesetround(FE_TONEAREST);
+    long nb = (n + B - 1) / B;
+    for (long b = 0; b < nb; ++b) {
+        long lo = b * (long)B;
+        long hi = lo + B < n ? lo + B : n;
+        float amax = 0.0f;
+        for (long i = lo; i < hi; ++i) {
+            float a = fabsf(x[i]);
+            if (a > amax) amax = a;
+        }
+        absmax[b] = amax;
+        float scale = amax > 0.0f ? 127.0f / amax : 0.0f;
+        for (long i = lo; i < hi; ++i) q[i] = amax > 0.0f ? quantize_one(x[i], scale) : 0;
+    }
+}
+
+/* x'[i] = (q[i] * absmax[block of i]) / 127 in fp32, left to right. */
+void orc_block_dequantize(const int8_t* q, const float* absmax, long n, int B, float* out) {
+    fesetround(FE_TONEAREST);
+    for (long i = 0; i < n; ++i) {
+        float t = (float)q[i] * absmax[i / B];
+        out[i] = t / 127.0f;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Group-wise int8 matmul: the vector-wise method with one normalisation    */
+/* constant per group of G consecutive inner-product indices instead of one */
+/* per whole vector (the granularity of nuQmm and ZeroQuant, which the      */
+/* scite report for nuQmm cites as finer than vector-wise; its GPTQ snippet */
+/* puts runs of consecutive weights under one constant).  G divides K.  The */
+/* outlier decomposition is unchanged: outlier columns are zero in the int8 */
+/* operand and go through the 16-bit product; a group whose every column is */
+/* an outlier has absmax 0.                                                  */
+/*   ra[m*ng + g] = max |X[m,k]| over k in group g, k not an outlier        */
+/*   ca[n*ng + g] = max |W[k,n]| over k in group g                          */
+/*   acc_g[m,n]   = sum over k in group g of Xq[m,k] * Wq[n,k] (exact)      */
+/*   y = fp16( sum_g acc_g * ra * ca / 16129 (fp32, ascending g) + o )      */
+/* With G = K every step is the vector-wise one, bit for bit.               */
+/* ------------------------------------------------------------------------ */
+
+void orc_quantize_rows_grouped(const uint16_t* X, int M, int K, int G, const int32_t* idx, int n_o,
+                               int8_t* Xq, float* ra, uint16_t* Xo) {
+    fesetround(FE_TONEAREST);
+    int ng = K / G;
+    unsigned char* is_out = (unsigned char*)calloc((size_t)K > 0 ? (size_t)K : 1, 1);
+    for (int j = 0; j < n_o; ++j) is_out[idx[j]] = 1;
+    for (int m = 0; m < M; ++m) {
+        const uint16_t* row = X + (size_t)m * K;
+        for (int g = 0; g < ng; ++g) {
+            float amax = 0.0f;
+            for (int k = g * G; k < (g + 1) * G; ++k) {
+                if (is_out[k]) continue;
+                float a = fabsf(orc_half_to_float(row[k]));
+                if (a > amax) amax = a;
+            }
+            ra[(size_t)m * ng + g] = amax;
+            float scale = amax > 0.0f ? 127.0f / amax : 0.0f;
+            for (int k = g * G; k < (g + 1) * G; ++k) {
+                int8_t q = 0;
+                if (!is_out[k] && amax > 0.0f) q = quantize_one(orc_half_to_float(row[k]), scale);
+                Xq[(size_t)m * K + k] = q;
+            }
+        }
+        for (int j = 0; j < n_o; ++j) Xo[(size_t)m * n_o + j] = row[idx[j]];
+    }
+    free(is_out);
+}
+
+void orc_quantize_weight_grouped(const uint16_t* W, int K, int N, int G, int8_t* Wq, float* ca) {
+    fesetround(FE_TONEAREST);
+    int ng = K / G;
+    for (int n = 0; n < N; ++n) {
+        for (int g = 0; g < ng; ++g) {
+            float amax = 0.0f;
+            for (int k = g * G; k < (g + 1) * G; ++k) {
+                float a = fabsf(orc_half_to_float(W[(size_t)k * N + n]));
+                if (a > amax) amax = a;
+            }
+            ca[(size_t)n * ng + g] = amax;
+            float scale = amax > 0.0f ? 127.0f / amax : 0.0f;
+            for (int k = g * G; k < (g + 1) * G; ++k) {
+                int8_t q = 0;
+                if (amax > 0.0f) q = quantize_one(orc_half_to_float(W[(size_t)k * N + n]), scale);
+                Wq[(size_t)n * K + k] = q;
+            }
+        }
+    }
+}
+
+/* Wo (n_o x N) for the group-wise weight: the kept fp16 row, else the row  */
+/* dequantised with its own group's constant, fp16((q * ca[n, k/G]) / 127). */
+void orc_gather_w_outlier_grouped(const uint16_t* W_keep, const int32_t* keep_idx, int n_keep,
+                                  const int8_t* Wq, const float* ca, int K, int N, int G,
+                                  const int32_t* idx, int n_o, uint16_t* Wo) {
+    fesetround(FE_TONEAREST);
+    int ng = K / G;
+    for (int j = 0; j < n_o; ++j) {
+        int k = idx[j];
+        int slot = -1;
+        for (int i = 0; i < n_keep; ++i)
+            if (keep_idx[i] == k) {
+                slot = i;
+                break;
+            }
+        for (int n = 0; n < N; ++n) {
+            uint16_t w;
+            if (slot >= 0) {
+                w = W_keep[(size_t)slot * N + n];
+            } else {
+                float t = (float)Wq[(size_t)n * K + k] * ca[(size_t)n * ng + k / G];
+                w = orc_float_to_half(t / 127.0f);
+            }
+            Wo[(size_t)j * N + n] = w;
+        }
+    }
+}
+
+/* acc_g (optional, M x N x ng) and Y (M x N) of the group-wise product;    */
+/* o (M x N fp32, may be NULL) is the 16-bit outlier product.  Returns 0,   */
+/* or -1 if a group sum does not fit int32.                                 */
+int orc_grouped_forward(const int8_t* Xq, const float* ra, const int8_t* Wq, const float* ca,
+                        const float* o, int M, int N, int K, int G, int32_t* acc_out, uint16_t* Y) {
+    fesetround(FE_TONEAREST);
+    int ng = K / G;
+    int overflow = 0;
+    for (int m = 0; m < M; ++m) {
+        const int8_t* a = Xq + (size_t)m * K;
+        for (int n = 0; n < N; ++n) {
+            const int8_t* b = Wq + (size_t)n * K;
+            float v = 0.0f;
+            for (int g = 0; g < ng; ++g) {
+                int64_t s = 0;
+                for (int k = g * G; k < (g + 1) * G; ++k) s += (int64_t)a[k] * (int64_t)b[k];
+                if (s > INT32_MAX || s < INT32_MIN) overflow = 1;
+                if (acc_out) acc_out[((size_t)m * N + n) * ng + g] = (int32_t)s;
+                float t = (float)(int32_t)s;
+                t = t * ra[(size_t)m * ng + g];
+                t = t * ca[(size_t)n * ng + g];
+                t = t / 16129.0f;
+                v = v + t;
+            }
+            v = v + (o ? o[(size_t)m * N + n] : 0.0f);
+            Y[(size_t)m * N + n] = orc_float_to_half(v);
+        }
+    }
+    return overflow ? -1 : 0;
 }

@@ -45,10 +45,55 @@ MUTATIONS = {
     "half_encode_truncates": ("float m = nearbyintf(ldexpf(a, 10 - e));", "float m = truncf(ldexpf(a, 10 - e));"),
 }
 
+# mistakes in the variants (block-wise codec, group-wise matmul)
+VARIANT_MUTATIONS = {
+    "block_short_by_one": ("long hi = lo + B < n ? lo + B : n;", "long hi = lo + B - 1 < n ? lo + B - 1 : n;"),
+    "block_absmax_whole_vector": ("for (long i = lo; i < hi; ++i) {\n            float a = fabsf(x[i]);",
+                                  "for (long i = 0; i < n; ++i) {\n            float a = fabsf(x[i]);"),
+    "block_dequant_over_128": ("out[i] = t / 127.0f;", "out[i] = t / 128.0f;"),
+    "block_dequant_next_constant": ("float t = (float)q[i] * absmax[i / B];",
+                                    "float t = (float)q[i] * absmax[(i + 1) / B < (n + B - 1) / B ? (i + 1) / B : i / B];"),
+    "grouped_x_absmax_whole_row": ("for (int k = g * G; k < (g + 1) * G; ++k) {\n                if (is_out[k]) continue;",
+                                   "for (int k = 0; k < K; ++k) {\n                if (is_out[k]) continue;"),
+    "grouped_outliers_in_absmax": ("                if (is_out[k]) continue;\n                float a", "                float a"),
+    "grouped_w_absmax_whole_column": ("for (int k = g * G; k < (g + 1) * G; ++k) {\n                float a = fabsf(orc_half_to_float(W[",
+                                      "for (int k = 0; k < K; ++k) {\n                float a = fabsf(orc_half_to_float(W["),
+    "grouped_epilogue_first_constant": ("t = t * ca[(size_t)n * ng + g];", "t = t * ca[(size_t)n * ng];"),
+    "grouped_sum_drops_last_group": ("v = v + t;\n            }", "if (g + 1 < ng || ng == 1) v = v + t;\n            }"),
+    "grouped_dequant_row_first_constant": ("ca[(size_t)n * ng + k / G]", "ca[(size_t)n * ng]"),
+}
+
+
+def _run(checks):
+    failed = []
+    for name, fn in checks.items():
+        try:
+            fn()
+        except Exception:  # noqa: BLE001 - any failure counts as caught
+            failed.append(name)
+    return failed
+
+
+def _variant_pin_suite():
+    """A fast subset of the variants' pins; return the names of those that fail."""
+    from tests import test_oracle_variant_pins as vp
+
+    checks = {
+        "block_golden": vp.test_block_worked_example_golden,
+        "block_isolation": vp.test_block_outlier_stays_in_its_block,
+        "block_integers": vp.test_block_integers_round_trip_exactly,
+        "grouped_one_group": lambda: vp.test_grouped_with_one_group_is_the_vectorwise_method(False),
+        "grouped_integers": vp.test_grouped_integer_inputs_give_the_exact_product,
+        "grouped_error_bound": vp.test_grouped_result_within_method_error_bound,
+    }
+    for seed in range(30):
+        checks[f"block_brute_force_{seed}"] = (lambda s=seed: vp.test_block_brute_force(s))
+        checks[f"grouped_brute_force_{seed}"] = (lambda s=seed: vp.test_grouped_brute_force_tiny(s))
+    return _run(checks)
+
 
 def _pin_suite():
     """Run a fast subset of the pins; return the names of those that fail."""
-    failed = []
     checks = {
         "half_decode": pins.test_half_to_float_exhaustive,
         "half_encode": pins.test_float_to_half_round_half_even,
@@ -64,20 +109,24 @@ def _pin_suite():
         checks[f"rule_exhaustive_{amax}"] = (lambda a=amax: pins.test_quantisation_rule_exhaustive(a))
     for seed in range(40):
         checks[f"brute_force_{seed}"] = (lambda s=seed: pins.test_brute_force_tiny(s))
-    for name, fn in checks.items():
-        try:
-            fn()
-        except Exception:  # noqa: BLE001 - any failure counts as caught
-            failed.append(name)
-    return failed
+    return _run(checks)
 
 
-@pytest.mark.parametrize("name", sorted(MUTATIONS))
-def test_planted_mistake_is_caught(name, tmp_path):
-    old, new = MUTATIONS[name]
+VARIANTS_MARKER = "Variants beyond the vector-wise matmul"
+
+
+def _mutated_suite_failures(old, new, suite, tmp_path, variant):
+    """Plant the mistake at the anchor's first occurrence, which must lie in
+    the vector-wise part of the source (or, for a variant, be the only one and
+    lie in the variants' part); return the pins that fail."""
     with open(oracle._SRC) as f:
         src = f.read()
-    assert src.count(old) >= 1, f"mutation anchor for {name} not found"
+    at, marker = src.find(old), src.find(VARIANTS_MARKER)
+    assert at >= 0 and marker >= 0, f"mutation anchor {old!r} not found"
+    if variant:
+        assert at > marker and src.count(old) == 1, f"variant anchor {old!r} must occur once, among the variants"
+    else:
+        assert at < marker, f"anchor {old!r} must first occur in the vector-wise part"
     mutated = src.replace(old, new, 1)
     c_path = os.path.join(tmp_path, "mut.c")
     so_path = os.path.join(tmp_path, "libmut.so")
@@ -86,11 +135,23 @@ def test_planted_mistake_is_caught(name, tmp_path):
     subprocess.run(["gcc", *oracle._CFLAGS, "-o", so_path, c_path, "-lm"], check=True)
     oracle._swap_library(so_path)
     try:
-        failed = _pin_suite()
+        return suite()
     finally:
         oracle._swap_library(None)
-    assert failed, f"planted mistake {name!r} passed every pin"
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, tmp_path):
+    old, new = MUTATIONS[name]
+    assert _mutated_suite_failures(old, new, _pin_suite, tmp_path, False), f"planted mistake {name!r} passed every pin"
+
+
+@pytest.mark.parametrize("name", sorted(VARIANT_MUTATIONS))
+def test_planted_variant_mistake_is_caught(name, tmp_path):
+    old, new = VARIANT_MUTATIONS[name]
+    assert _mutated_suite_failures(old, new, _variant_pin_suite, tmp_path, True), f"planted mistake {name!r} passed every pin"
 
 
 def test_unmutated_oracle_passes_suite():
     assert _pin_suite() == []
+    assert _variant_pin_suite() == []
