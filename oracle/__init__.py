@@ -24,7 +24,10 @@ raw 16-bit patterns.  Each wrapper names the passage it follows:
   (blocks normalised by their own maximum, an 8-bit index per value);
 * group-wise matmul -- the scite report for nuQmm (nuQmm / ZeroQuant use one
   constant per group, finer than vector-wise; GPTQ's grouping of consecutive
-  weights).
+  weights);
+* 4-bit weight-only product -- the talk's "4-Bit Inference" and the axolotl
+  page's "Impact of Precision and Parameter Count" (weight loading dominates
+  inference, so bits per weight set its time).
 """
 from __future__ import annotations
 
@@ -95,6 +98,12 @@ def _setup(lib):
     lib.orc_gather_w_outlier_grouped.restype = None
     lib.orc_grouped_forward.argtypes = [P, P, P, P, P, I, I, I, I, P, P]
     lib.orc_grouped_forward.restype = I
+    lib.orc_double_to_half.argtypes = [ctypes.c_double]
+    lib.orc_double_to_half.restype = ctypes.c_uint16
+    lib.orc_quantize_weight_int4.argtypes = [P, I, I, I, P, P]
+    lib.orc_quantize_weight_int4.restype = None
+    lib.orc_int4_product.argtypes = [P, P, P, I, I, I, I, P]
+    lib.orc_int4_product.restype = None
     return lib
 
 
@@ -397,3 +406,36 @@ def forward_grouped(X: np.ndarray, prep: dict, threshold: float) -> dict:
     o = outlier_gemm(Xo, Wo)
     acc, Y = grouped_product(Xq, ra, prep["wq"], prep["ca"], G, o)
     return {"idx": idx, "xq": Xq, "ra": ra, "xo": Xo, "acc": acc, "wo": Wo, "o": o, "y": Y}
+
+
+# --------------------------------------------------------------------------
+# 4-bit weight-only product
+# --------------------------------------------------------------------------
+
+def double_to_half(x: float) -> int:
+    return int(_load().orc_double_to_half(float(x)))
+
+
+def quantize_weight_int4(W: np.ndarray, G: int):
+    """W (K x N fp16) -> (codes int8 N x K in [-7, 7], ca float32 N x K/G)."""
+    wb = _bits(W)
+    K, N = wb.shape
+    assert G >= 1 and K % G == 0
+    q = np.zeros((N, K), dtype=np.int8)
+    ca = np.zeros((N, K // G), dtype=np.float32)
+    _load().orc_quantize_weight_int4(_ptr(wb), K, N, int(G), _ptr(q), _ptr(ca))
+    return q, ca
+
+
+def int4_product(X: np.ndarray, q: np.ndarray, ca: np.ndarray, G: int) -> np.ndarray:
+    """Y (M x N fp16) = X (M x K fp16) times the dequantised 4-bit weight."""
+    xb = _bits(X)
+    M, K = xb.shape
+    q = _c(q, np.int8)
+    N = q.shape[0]
+    assert q.shape[1] == K and K % G == 0
+    ca = _c(ca, np.float32)
+    assert ca.shape == (N, K // G)
+    Y = np.zeros((M, N), dtype=np.uint16)
+    _load().orc_int4_product(_ptr(xb), _ptr(q), _ptr(ca), M, N, K, int(G), _ptr(Y))
+    return Y.view(np.float16)

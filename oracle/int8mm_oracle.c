@@ -35,10 +35,11 @@
  *     else from the dequantised int8 row fp16(q * ca / 127);
  *   - y = fp16( (float)acc * ra[m] * ca[n] / 16129 + o ), left to right.
  *
- * Two variants follow the vector-wise matmul at the end of the file, with
- * the same per-value rule: a block-wise linear 8-bit codec of an fp32 vector
- * and the group-wise matmul (one constant per group of G consecutive inner
- * indices).  The GPU library does not implement them yet.
+ * Three variants follow the vector-wise matmul at the end of the file, with
+ * the same per-value rule: a block-wise linear 8-bit codec of an fp32 vector,
+ * the group-wise matmul (one constant per group of G consecutive inner
+ * indices) and a 4-bit weight-only product.  The GPU library does not
+ * implement them yet.
  *
  * Build: gcc -O2 -ffp-contract=off (no fast-math), -pthread.
  */
@@ -507,4 +508,79 @@ int orc_grouped_forward(const int8_t* Xq, const float* ra, const int8_t* Wq, con
         }
     }
     return overflow ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* 4-bit weight-only product for decode-sized X.  Inference is bound by     */
+/* loading the weights, so fewer bits per weight cut its time at the same   */
+/* parameter count (video of the talk, "4-Bit Inference"; axolotl page,     */
+/* "Impact of Precision and Parameter Count").  Weights get linear 4-bit    */
+/* codes in [-7, 7] with one constant per output column and group of G      */
+/* consecutive k (G divides K), by the same rule as the 8-bit codes with 7  */
+/* in place of 127; X stays fp16.                                           */
+/*   ca[n*ng + g] = max |W[k,n]| over k in group g                          */
+/*   q[n*K + k]   = clamp(round-half-even(RN32(W[k,n] * RN32(7/ca))), +-7)  */
+/*   w'           = RN32(RN32(q * ca) / 7)                                  */
+/*   Y[m,n]       = fp16( sum_k x[m,k] * w'[k,n] ), summed in double        */
+/* ------------------------------------------------------------------------ */
+
+/* Round-to-nearest-even conversion of a binary64 value to binary16 bits. */
+uint16_t orc_double_to_half(double f) {
+    uint16_t sign = signbit(f) ? 0x8000u : 0u;
+    if (isnan(f)) return (uint16_t)(sign | 0x7e00u);
+    double a = fabs(f);
+    if (a >= 65520.0) return (uint16_t)(sign | 0x7c00u);
+    if (a < ldexp(1.0, -14)) return (uint16_t)(sign | (uint16_t)nearbyint(ldexp(a, 24)));
+    int e;
+    frexp(a, &e);
+    e -= 1;
+    double m = nearbyint(ldexp(a, 10 - e));
+    if (m == 2048.0) {
+        m = 1024.0;
+        e += 1;
+    }
+    if (e + 15 >= 31) return (uint16_t)(sign | 0x7c00u);
+    return (uint16_t)(sign | (uint16_t)((e + 15) << 10) | (uint16_t)((int)m - 1024));
+}
+
+void orc_quantize_weight_int4(const uint16_t* W, int K, int N, int G, int8_t* q, float* ca) {
+    fesetround(FE_TONEAREST);
+    int ng = K / G;
+    for (int n = 0; n < N; ++n) {
+        for (int g = 0; g < ng; ++g) {
+            float amax = 0.0f;
+            for (int k = g * G; k < (g + 1) * G; ++k) {
+                float a = fabsf(orc_half_to_float(W[(size_t)k * N + n]));
+                if (a > amax) amax = a;
+            }
+            ca[(size_t)n * ng + g] = amax;
+            float scale = amax > 0.0f ? 7.0f / amax : 0.0f;
+            for (int k = g * G; k < (g + 1) * G; ++k) {
+                int8_t c = 0;
+                if (amax > 0.0f) {
+                    float r = nearbyintf(orc_half_to_float(W[(size_t)k * N + n]) * scale);
+                    if (r > 7.0f) r = 7.0f;
+                    if (r < -7.0f) r = -7.0f;
+                    c = (int8_t)r;
+                }
+                q[(size_t)n * K + k] = c;
+            }
+        }
+    }
+}
+
+void orc_int4_product(const uint16_t* X, const int8_t* q, const float* ca, int M, int N, int K, int G,
+                      uint16_t* Y) {
+    fesetround(FE_TONEAREST);
+    int ng = K / G;
+    for (int m = 0; m < M; ++m)
+        for (int n = 0; n < N; ++n) {
+            double s = 0.0;
+            for (int k = 0; k < K; ++k) {
+                float t = (float)q[(size_t)n * K + k] * ca[(size_t)n * ng + k / G];
+                float w = t / 7.0f;
+                s += (double)orc_half_to_float(X[(size_t)m * K + k]) * (double)w;
+            }
+            Y[(size_t)m * N + n] = orc_double_to_half(s);
+        }
 }

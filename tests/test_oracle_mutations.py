@@ -45,7 +45,7 @@ MUTATIONS = {
     "half_encode_truncates": ("float m = nearbyintf(ldexpf(a, 10 - e));", "float m = truncf(ldexpf(a, 10 - e));"),
 }
 
-# mistakes in the variants (block-wise codec, group-wise matmul)
+# mistakes in the variants (block-wise codec, group-wise matmul, 4-bit product)
 VARIANT_MUTATIONS = {
     "block_short_by_one": ("long hi = lo + B < n ? lo + B : n;", "long hi = lo + B - 1 < n ? lo + B - 1 : n;"),
     "block_absmax_whole_vector": ("for (long i = lo; i < hi; ++i) {\n            float a = fabsf(x[i]);",
@@ -56,11 +56,23 @@ VARIANT_MUTATIONS = {
     "grouped_x_absmax_whole_row": ("for (int k = g * G; k < (g + 1) * G; ++k) {\n                if (is_out[k]) continue;",
                                    "for (int k = 0; k < K; ++k) {\n                if (is_out[k]) continue;"),
     "grouped_outliers_in_absmax": ("                if (is_out[k]) continue;\n                float a", "                float a"),
-    "grouped_w_absmax_whole_column": ("for (int k = g * G; k < (g + 1) * G; ++k) {\n                float a = fabsf(orc_half_to_float(W[",
-                                      "for (int k = 0; k < K; ++k) {\n                float a = fabsf(orc_half_to_float(W["),
+    "grouped_w_absmax_whole_column": (
+        "for (int k = g * G; k < (g + 1) * G; ++k) {\n                float a = fabsf(orc_half_to_float(W[(size_t)k * N + n]));"
+        "\n                if (a > amax) amax = a;\n            }\n            ca[(size_t)n * ng + g] = amax;\n"
+        "            float scale = amax > 0.0f ? 127.0f",
+        "for (int k = 0; k < K; ++k) {\n                float a = fabsf(orc_half_to_float(W[(size_t)k * N + n]));"
+        "\n                if (a > amax) amax = a;\n            }\n            ca[(size_t)n * ng + g] = amax;\n"
+        "            float scale = amax > 0.0f ? 127.0f"),
     "grouped_epilogue_first_constant": ("t = t * ca[(size_t)n * ng + g];", "t = t * ca[(size_t)n * ng];"),
     "grouped_sum_drops_last_group": ("v = v + t;\n            }", "if (g + 1 < ng || ng == 1) v = v + t;\n            }"),
-    "grouped_dequant_row_first_constant": ("ca[(size_t)n * ng + k / G]", "ca[(size_t)n * ng]"),
+    "grouped_dequant_row_first_constant": ("Wq[(size_t)n * K + k] * ca[(size_t)n * ng + k / G]",
+                                           "Wq[(size_t)n * K + k] * ca[(size_t)n * ng]"),
+    "int4_clamp_at_6": ("if (r > 7.0f) r = 7.0f;", "if (r > 6.0f) r = 6.0f;"),
+    "int4_scale_over_8": ("float scale = amax > 0.0f ? 7.0f / amax : 0.0f;", "float scale = amax > 0.0f ? 8.0f / amax : 0.0f;"),
+    "int4_dequant_over_8": ("float w = t / 7.0f;", "float w = t / 8.0f;"),
+    "int4_dequant_first_group": ("ca[(size_t)n * ng + k / G];\n                float w", "ca[(size_t)n * ng];\n                float w"),
+    "int4_sum_through_fp32": ("Y[(size_t)m * N + n] = orc_double_to_half(s);", "Y[(size_t)m * N + n] = orc_float_to_half((float)s);"),
+    "int4_half_round_truncates": ("double m = nearbyint(ldexp(a, 10 - e));", "double m = trunc(ldexp(a, 10 - e));"),
 }
 
 
@@ -85,10 +97,15 @@ def _variant_pin_suite():
         "grouped_one_group": lambda: vp.test_grouped_with_one_group_is_the_vectorwise_method(False),
         "grouped_integers": vp.test_grouped_integer_inputs_give_the_exact_product,
         "grouped_error_bound": vp.test_grouped_result_within_method_error_bound,
+        "double_to_half": vp.test_double_to_half_rounds_once,
+        "int4_single_rounding": vp.test_int4_rounds_the_sum_once,
+        "int4_bound": vp.test_int4_absmax_maps_to_7_and_error_within_half_step,
+        "int4_integers": vp.test_int4_integer_weights_are_exact,
     }
     for seed in range(30):
         checks[f"block_brute_force_{seed}"] = (lambda s=seed: vp.test_block_brute_force(s))
         checks[f"grouped_brute_force_{seed}"] = (lambda s=seed: vp.test_grouped_brute_force_tiny(s))
+        checks[f"int4_brute_force_{seed}"] = (lambda s=seed: vp.test_int4_brute_force_tiny(s))
     return _run(checks)
 
 

@@ -13,7 +13,12 @@ without trusting the oracle:
   method bit for bit, a brute force in exact rationals, integer inputs that
   give the exact integer product, G = 1 reproduces the fp32 product, the
   method's error bound per group, and finer groups lowering the error on
-  weights with large entries.
+  weights with large entries;
+* the 4-bit weight-only product (the talk's "4-Bit Inference"; axolotl page,
+  "Impact of Precision and Parameter Count") -- correctly rounded double to
+  fp16, a brute force in exact rationals, a sum that must be rounded to fp16
+  once, +-absmax -> +-7 with the half-step bound, and integer weights that
+  give the exact product.
 """
 from __future__ import annotations
 
@@ -365,3 +370,117 @@ def test_finer_groups_lower_the_error_on_uneven_weights():
         y = oracle.forward_grouped(X, prep, math.inf)["y"].astype(np.float64)
         err[G] = float(np.sqrt(np.mean((y - exact) ** 2)))
     assert err[32] < err[128] < err[1024]
+
+
+# --------------------------------------------------------------------------
+# 4-bit weight-only product
+# --------------------------------------------------------------------------
+
+def test_double_to_half_rounds_once():
+    rng = np.random.default_rng(30)
+    h = np.arange(0x0001, 0x7bff, 5, dtype=np.uint16)
+    lo = h.view(np.float16).astype(np.float64)
+    hi = (h + 1).view(np.float16).astype(np.float64)
+    mid = (lo + hi) / 2
+    vals = list(mid) + list(mid * (1 + 2.0 ** -40)) + list(mid * (1 - 2.0 ** -40))
+    vals += list(rng.standard_normal(3000) * 300.0) + [0.0, -0.0, 65504.0, 65519.99, 65520.0, 1e300, 2.0 ** -25,
+                                                        2.0 ** -25 * (1 + 2.0 ** -40), 3 * 2.0 ** -26]
+    for v in vals:
+        with np.errstate(over="ignore"):
+            want = int(np.array(v, dtype=np.float64).astype(np.float16).view(np.uint16))
+        assert oracle.double_to_half(v) == want, (v, hex(want))
+        if np.isfinite(v) and abs(v) < 65520:
+            r = rn16(Fraction(v))
+            assert np.float16(r).view(np.uint16) == want or (r == 0 and (want & 0x7FFF) == 0)
+
+
+def int4_brute_force(X: np.ndarray, W: np.ndarray, G: int):
+    M, K = X.shape
+    N = W.shape[1]
+    xs = [[Fraction(float(v)) for v in row] for row in X.astype(np.float64)]
+    ws = [[Fraction(float(v)) for v in row] for row in W.astype(np.float64)]
+    q = [[0] * K for _ in range(N)]
+    ca = [[Fraction(0)] * (K // G) for _ in range(N)]
+    for n in range(N):
+        for g in range(K // G):
+            cols = range(g * G, (g + 1) * G)
+            a = max(abs(ws[k][n]) for k in cols)
+            ca[n][g] = a
+            if a == 0:
+                continue
+            s = rn32(Fraction(7) / a)
+            for k in cols:
+                q[n][k] = max(-7, min(7, round(rn32(ws[k][n] * s))))
+    wd = [[rn32(rn32(q[n][k] * ca[n][k // G]) / 7) for k in range(K)] for n in range(N)]
+    y = [[rn16(sum(xs[m][k] * wd[n][k] for k in range(K))) for n in range(N)] for m in range(M)]
+    return q, [[float(v) for v in r] for r in ca], y
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_int4_brute_force_tiny(seed):
+    rng = np.random.default_rng(2000 + seed)
+    G = int(rng.choice([1, 2, 4, 5]))
+    K = G * int(rng.integers(1, 4))
+    M, N = (int(v) for v in rng.integers(1, 7, size=2))
+    X = (rng.standard_normal((M, K)) * rng.choice([0.5, 4.0])).astype(np.float16)
+    W = (rng.standard_normal((K, N)) * rng.choice([0.02, 1.0])).astype(np.float16)
+    if rng.random() < 0.3:
+        W[:, int(rng.integers(0, N))] = 0
+    q, ca = oracle.quantize_weight_int4(W, G)
+    bq, bca, by = int4_brute_force(X, W, G)
+    assert q.tolist() == bq
+    assert ca.astype(np.float64).tolist() == bca
+    y = oracle.int4_product(X, q, ca, G)
+    assert np.array_equal(y.astype(np.float64), np.array(by, dtype=np.float64).reshape(y.shape))
+
+
+def test_int4_rounds_the_sum_once():
+    """1 + 2^-11 + 2^-24 lies just above the midpoint of 1 and 1 + 2^-10: one
+    rounding to fp16 gives 1 + 2^-10 (a detour through fp32 would make it a tie
+    and give 1)."""
+    X = np.array([[1.0, 2.0 ** -11, 2.0 ** -24, 0.0]], dtype=np.float16)
+    W = np.array([[1.0], [1.0], [1.0], [7.0]], dtype=np.float16)
+    q, ca = oracle.quantize_weight_int4(W, 4)
+    assert q[:, :].tolist() == [[1, 1, 1, 7]] and ca.tolist() == [[7.0]]
+    assert float(oracle.int4_product(X, q, ca, 4)[0, 0]) == 1.0 + 2.0 ** -10
+
+
+def test_int4_absmax_maps_to_7_and_error_within_half_step():
+    X, W, _ = synth.make_case(8, 1024, 96, seed=31)
+    W = W.numpy()
+    G = 128
+    q, ca = oracle.quantize_weight_int4(W, G)
+    assert np.abs(q.astype(np.int32)).max() <= 7
+    wf = W.astype(np.float64)
+    for n in range(0, 96, 7):
+        for g in range(1024 // G):
+            blk = wf[g * G:(g + 1) * G, n]
+            i = int(np.argmax(np.abs(blk)))
+            assert abs(blk[i]) == ca[n, g]
+            assert q[n, g * G + i] == (7 if blk[i] > 0 else -7)
+    step = np.repeat(ca.astype(np.float64), G, axis=1).T / 7.0  # K x N
+    wd = q.T.astype(np.float64) * np.repeat(ca.astype(np.float64), G, axis=1).T / 7.0
+    assert np.all(np.abs(wf - wd) <= step / 2 * (1 + 2.0 ** -20))
+    # Y against the exact product: the weight half-steps plus the fp16 rounding
+    X = X.numpy().astype(np.float64)
+    y = oracle.int4_product(X.astype(np.float16), q, ca, G).astype(np.float64)
+    exact = X @ wf
+    # weight half-steps, the fp32 roundings of w', the final fp16 rounding
+    bound = (np.abs(X) @ (step / 2 * (1 + 2.0 ** -20)) + (np.abs(X) @ np.abs(wd)) * 2.0 ** -22
+             + np.abs(y) * 2.0 ** -11 + 2.0 ** -25)
+    assert np.all(np.abs(y - exact) <= bound)
+
+
+def test_int4_integer_weights_are_exact():
+    rng = np.random.default_rng(32)
+    K, N, G = 32, 9, 8
+    W = rng.integers(-7, 8, size=(K, N)).astype(np.float16)
+    for g in range(K // G):
+        W[g * G + rng.integers(0, G, N), np.arange(N)] = 7 * rng.choice([-1, 1], N)
+    q, ca = oracle.quantize_weight_int4(W, G)
+    assert np.all(ca == 7.0)
+    assert np.array_equal(q.T.astype(np.float16), W)
+    X = rng.integers(-16, 17, size=(3, K)).astype(np.float16)
+    exact = X.astype(np.int64) @ W.astype(np.int64)
+    assert np.array_equal(oracle.int4_product(X, q, ca, G).astype(np.float64),
+                          exact.astype(np.float16).astype(np.float64))
