@@ -137,13 +137,47 @@ KERNEL_SOURCES = {
 }
 
 
+def strip_comments(src: str) -> str:
+    """C/C++ source with every run of whitespace and // or /* */ comments
+    outside string and character literals reduced to one space (literals kept
+    as they are), so that editing a comment or the layout does not count as a
+    change of the kernel."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif c.isspace() or src.startswith("//", i) or src.startswith("/*", i):
+            # a run of whitespace and comments becomes one space
+            while i < n:
+                if src[i].isspace():
+                    i += 1
+                elif src.startswith("//", i):
+                    j = src.find("\n", i)
+                    i = n if j < 0 else j
+                elif src.startswith("/*", i):
+                    j = src.find("*/", i + 2)
+                    i = n if j < 0 else j + 2
+                else:
+                    break
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return "".join(out)
+
+
 def kernel_source_sha(kernel: str) -> str:
-    """Hash of the source files a kernel is compiled from."""
+    """Hash of the code (comments stripped) of the files a kernel is compiled from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "int8_quantized_matmul_02_b200", "csrc")
     for f in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            h.update(strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
