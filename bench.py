@@ -168,7 +168,7 @@ def strip_comments(src: str) -> str:
         else:
             out.append(c)
             i += 1
-    return "".join(out)
+    return "".join(out).strip()
 
 
 def kernel_source_sha(kernel: str) -> str:
