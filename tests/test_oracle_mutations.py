@@ -76,17 +76,21 @@ VARIANT_MUTATIONS = {
 }
 
 
-def _run(checks):
+def _run(checks, first_only=False):
+    """Run the checks in order; return the names of those that fail (only the
+    first one when first_only: a planted mistake is caught by any pin)."""
     failed = []
     for name, fn in checks.items():
         try:
             fn()
         except Exception:  # noqa: BLE001 - any failure counts as caught
             failed.append(name)
+            if first_only:
+                break
     return failed
 
 
-def _variant_pin_suite():
+def _variant_pin_suite(first_only=False):
     """A fast subset of the variants' pins; return the names of those that fail."""
     from tests import test_oracle_variant_pins as vp
 
@@ -106,14 +110,13 @@ def _variant_pin_suite():
         checks[f"block_brute_force_{seed}"] = (lambda s=seed: vp.test_block_brute_force(s))
         checks[f"grouped_brute_force_{seed}"] = (lambda s=seed: vp.test_grouped_brute_force_tiny(s))
         checks[f"int4_brute_force_{seed}"] = (lambda s=seed: vp.test_int4_brute_force_tiny(s))
-    return _run(checks)
+    return _run(checks, first_only)
 
 
-def _pin_suite():
-    """Run a fast subset of the pins; return the names of those that fail."""
+def _pin_suite(first_only=False):
+    """Run a fast subset of the pins, cheapest first; return the names of
+    those that fail."""
     checks = {
-        "half_decode": pins.test_half_to_float_exhaustive,
-        "half_encode": pins.test_float_to_half_round_half_even,
         "worked_example": pins.test_worked_example_golden,
         "threshold_equality": pins.test_value_exactly_at_threshold_is_outlier,
         "absmax_127": pins.test_absmax_maps_to_127,
@@ -122,11 +125,13 @@ def _pin_suite():
         "error_bound": pins.test_result_within_method_error_bound,
         "dequantised_rows": pins.test_dequantised_outlier_rows_when_not_kept,
     }
-    for amax in (5.99609375, 3.140625, 40.96875, 0.46044921875, 1.5947265625):
-        checks[f"rule_exhaustive_{amax}"] = (lambda a=amax: pins.test_quantisation_rule_exhaustive(a))
     for seed in range(40):
         checks[f"brute_force_{seed}"] = (lambda s=seed: pins.test_brute_force_tiny(s))
-    return _run(checks)
+    checks["half_decode"] = pins.test_half_to_float_exhaustive
+    checks["half_encode"] = pins.test_float_to_half_round_half_even
+    for amax in (5.99609375, 3.140625, 40.96875, 0.46044921875, 1.5947265625):
+        checks[f"rule_exhaustive_{amax}"] = (lambda a=amax: pins.test_quantisation_rule_exhaustive(a))
+    return _run(checks, first_only)
 
 
 VARIANTS_MARKER = "Variants beyond the vector-wise matmul"
@@ -160,13 +165,15 @@ def _mutated_suite_failures(old, new, suite, tmp_path, variant):
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_planted_mistake_is_caught(name, tmp_path):
     old, new = MUTATIONS[name]
-    assert _mutated_suite_failures(old, new, _pin_suite, tmp_path, False), f"planted mistake {name!r} passed every pin"
+    suite = lambda: _pin_suite(first_only=True)  # noqa: E731
+    assert _mutated_suite_failures(old, new, suite, tmp_path, False), f"planted mistake {name!r} passed every pin"
 
 
 @pytest.mark.parametrize("name", sorted(VARIANT_MUTATIONS))
 def test_planted_variant_mistake_is_caught(name, tmp_path):
     old, new = VARIANT_MUTATIONS[name]
-    assert _mutated_suite_failures(old, new, _variant_pin_suite, tmp_path, True), f"planted mistake {name!r} passed every pin"
+    suite = lambda: _variant_pin_suite(first_only=True)  # noqa: E731
+    assert _mutated_suite_failures(old, new, suite, tmp_path, True), f"planted mistake {name!r} passed every pin"
 
 
 def test_unmutated_oracle_passes_suite():
