@@ -34,8 +34,10 @@
  *   - fp16 tensors are passed as pointers to IEEE binary16 bit patterns
  *     (uint16_t); all matrices are row-major and densely packed.
  *   - "device" pointers point to memory of the current CUDA device; the
- *     caller allocates and owns all memory.  The library allocates nothing
- *     on the device and keeps no global state between calls.
+ *     caller allocates and owns all memory.  The library calls no device
+ *     allocator.  Between calls it keeps only a per-device cache of device
+ *     properties on the host and, for int8mm_forward_decode_noalloc alone,
+ *     the static scratch array described with that function.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Calls are stream-ordered and do not synchronise the host,
  *     except where a function says so.
