@@ -104,6 +104,10 @@ def _setup(lib):
     lib.orc_quantize_weight_int4.restype = None
     lib.orc_int4_product.argtypes = [P, P, P, I, I, I, I, P]
     lib.orc_int4_product.restype = None
+    lib.orc_grouped_points.argtypes = [P, P, P, P, P, P, I, I, I, I, P, P, I, P, P]
+    lib.orc_grouped_points.restype = I
+    lib.orc_int4_points.argtypes = [P, P, P, I, I, P, P, I, P]
+    lib.orc_int4_points.restype = None
     return lib
 
 
@@ -397,6 +401,26 @@ def grouped_product(Xq, ra, Wq, ca, G: int, o=None):
     return acc, Y.view(np.float16)
 
 
+def forward_grouped_points(steps: dict, prep: dict, pm, pn):
+    """acc_g (npts x K/G) and Y at the points (pm[i], pn[i]) from the X-side
+    results of the group-wise forward (xq, ra, xo, wo)."""
+    G = prep["G"]
+    pm = _c(pm, np.int32)
+    pn = _c(pn, np.int32)
+    Xq = _c(steps["xq"], np.int8)
+    K = Xq.shape[1]
+    xo = _bits(steps["xo"])
+    wo = _bits(steps["wo"])
+    acc = np.zeros((pm.size, K // G), dtype=np.int32)
+    y = np.zeros(pm.size, dtype=np.uint16)
+    rc = _load().orc_grouped_points(_ptr(Xq), _ptr(_c(steps["ra"], np.float32)), _ptr(_c(prep["wq"], np.int8)),
+                                    _ptr(_c(prep["ca"], np.float32)), _ptr(xo), _ptr(wo), K, prep["N"], G,
+                                    xo.shape[1], _ptr(pm), _ptr(pn), pm.size, _ptr(acc), _ptr(y))
+    if rc != 0:
+        raise OverflowError("a group sum does not fit int32")
+    return acc, y.view(np.float16)
+
+
 def forward_grouped(X: np.ndarray, prep: dict, threshold: float) -> dict:
     """The group-wise forward pass; returns every intermediate and Y."""
     G = prep["G"]
@@ -439,3 +463,15 @@ def int4_product(X: np.ndarray, q: np.ndarray, ca: np.ndarray, G: int) -> np.nda
     Y = np.zeros((M, N), dtype=np.uint16)
     _load().orc_int4_product(_ptr(xb), _ptr(q), _ptr(ca), M, N, K, int(G), _ptr(Y))
     return Y.view(np.float16)
+
+
+def int4_points(X: np.ndarray, q: np.ndarray, ca: np.ndarray, G: int, pm, pn) -> np.ndarray:
+    """Y of the 4-bit weight-only product at the points (pm[i], pn[i])."""
+    xb = _bits(X)
+    K = xb.shape[1]
+    q = _c(q, np.int8)
+    pm = _c(pm, np.int32)
+    pn = _c(pn, np.int32)
+    y = np.zeros(pm.size, dtype=np.uint16)
+    _load().orc_int4_points(_ptr(xb), _ptr(q), _ptr(_c(ca, np.float32)), K, int(G), _ptr(pm), _ptr(pn), pm.size, _ptr(y))
+    return y.view(np.float16)

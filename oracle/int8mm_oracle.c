@@ -584,3 +584,50 @@ void orc_int4_product(const uint16_t* X, const int8_t* q, const float* ca, int M
             Y[(size_t)m * N + n] = orc_double_to_half(s);
         }
 }
+
+/* The group-wise product at a list of (m, n) points: acc_g (npts x ng) and */
+/* Y, the same arithmetic as orc_grouped_forward.  Returns 0, or -1 if a    */
+/* group sum does not fit int32.                                            */
+int orc_grouped_points(const int8_t* Xq, const float* ra, const int8_t* Wq, const float* ca,
+                       const uint16_t* Xo, const uint16_t* Wo, int K, int N, int G, int n_o,
+                       const int32_t* pm, const int32_t* pn, int npts, int32_t* acc_out,
+                       uint16_t* y_out) {
+    fesetround(FE_TONEAREST);
+    int ng = K / G;
+    int overflow = 0;
+    for (int p = 0; p < npts; ++p) {
+        const int8_t* a = Xq + (size_t)pm[p] * K;
+        const int8_t* b = Wq + (size_t)pn[p] * K;
+        float v = 0.0f;
+        for (int g = 0; g < ng; ++g) {
+            int64_t s = 0;
+            for (int k = g * G; k < (g + 1) * G; ++k) s += (int64_t)a[k] * (int64_t)b[k];
+            if (s > INT32_MAX || s < INT32_MIN) overflow = 1;
+            acc_out[(size_t)p * ng + g] = (int32_t)s;
+            float t = (float)(int32_t)s;
+            t = t * ra[(size_t)pm[p] * ng + g];
+            t = t * ca[(size_t)pn[p] * ng + g];
+            t = t / 16129.0f;
+            v = v + t;
+        }
+        v = v + outlier_dot(Xo, Wo, N, n_o, pm[p], pn[p]);
+        y_out[p] = orc_float_to_half(v);
+    }
+    return overflow ? -1 : 0;
+}
+
+/* The 4-bit weight-only product at a list of (m, n) points. */
+void orc_int4_points(const uint16_t* X, const int8_t* q, const float* ca, int K, int G, const int32_t* pm,
+                     const int32_t* pn, int npts, uint16_t* y_out) {
+    fesetround(FE_TONEAREST);
+    int ng = K / G;
+    for (int p = 0; p < npts; ++p) {
+        double s = 0.0;
+        for (int k = 0; k < K; ++k) {
+            float t = (float)q[(size_t)pn[p] * K + k] * ca[(size_t)pn[p] * ng + k / G];
+            float w = t / 7.0f;
+            s += (double)orc_half_to_float(X[(size_t)pm[p] * K + k]) * (double)w;
+        }
+        y_out[p] = orc_double_to_half(s);
+    }
+}

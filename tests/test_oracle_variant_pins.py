@@ -484,3 +484,29 @@ def test_int4_integer_weights_are_exact():
     exact = X.astype(np.int64) @ W.astype(np.int64)
     assert np.array_equal(oracle.int4_product(X, q, ca, G).astype(np.float64),
                           exact.astype(np.float16).astype(np.float64))
+
+
+# --------------------------------------------------------------------------
+# sampled points (the form the full-size parity checks use)
+# --------------------------------------------------------------------------
+
+def test_grouped_points_match_the_full_product():
+    X, W, keep = synth.make_case(70, 384, 90, n_seed=3, seed=33)
+    X = X.numpy()
+    W = W.numpy()
+    prep = oracle.prepare_weight_grouped(W, keep[:1], 64)
+    r = oracle.forward_grouped(X, prep, 6.0)
+    pm, pn = synth.sample_points(70, 90, 150, seed=3, tiles=((32, 32),))
+    acc, y = oracle.forward_grouped_points(r, prep, pm, pn)
+    assert np.array_equal(acc, r["acc"][pm, pn])
+    assert np.array_equal(y.view(np.uint16), r["y"][pm, pn].view(np.uint16))
+
+
+def test_int4_points_match_the_full_product():
+    X, W, _ = synth.make_case(9, 512, 80, seed=34)
+    X = X.numpy()
+    q, ca = oracle.quantize_weight_int4(W.numpy(), 128)
+    y_full = oracle.int4_product(X, q, ca, 128)
+    pm, pn = synth.sample_points(9, 80, 100, seed=4, tiles=((8, 16),))
+    y = oracle.int4_points(X, q, ca, 128, pm, pn)
+    assert np.array_equal(y.view(np.uint16), y_full[pm, pn].view(np.uint16))
