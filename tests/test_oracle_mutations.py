@@ -69,7 +69,8 @@ VARIANT_MUTATIONS = {
                                            "Wq[(size_t)n * K + k] * ca[(size_t)n * ng]"),
     "int4_clamp_at_6": ("if (r > 7.0f) r = 7.0f;", "if (r > 6.0f) r = 6.0f;"),
     "int4_scale_over_8": ("float scale = amax > 0.0f ? 7.0f / amax : 0.0f;", "float scale = amax > 0.0f ? 8.0f / amax : 0.0f;"),
-    "int4_dequant_over_8": ("float w = t / 7.0f;", "float w = t / 8.0f;"),
+    "int4_dequant_over_8": ("float w = t / 7.0f;\n                s += (double)orc_half_to_float(X[(size_t)m * K + k])",
+                            "float w = t / 8.0f;\n                s += (double)orc_half_to_float(X[(size_t)m * K + k])"),
     "int4_dequant_first_group": ("ca[(size_t)n * ng + k / G];\n                float w", "ca[(size_t)n * ng];\n                float w"),
     "int4_sum_through_fp32": ("Y[(size_t)m * N + n] = orc_double_to_half(s);", "Y[(size_t)m * N + n] = orc_float_to_half((float)s);"),
     "int4_half_round_truncates": ("double m = nearbyint(ldexp(a, 10 - e));", "double m = trunc(ldexp(a, 10 - e));"),
