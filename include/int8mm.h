@@ -6,16 +6,16 @@
  * feed-forward and attention-projection layers of a transformer, as a
  * two-part procedure --
  *   1. vector-wise quantisation: one normalisation constant per row of X and
- *      one per output column of W ("separate normalization constants for each
- *      inner product");
+ *      one per output column of W (each inner product gets its own pair of
+ *      constants);
  *   2. mixed-precision decomposition: the outlier feature dimensions of X go
  *      to a 16-bit matmul, everything else is multiplied in 8 bit.
  * Outliers are feature columns of the input batch (axolotl
  * "llama3-model-quantization", "Understanding Outliers in Transformer
  * Models"); quantisation normalises by the absolute maximum ("Key Points") and
  * rounds to the nearest level (scite report for nuQmm, which quotes LLM.int8()
- * as RTN); a 16/32-bit checkpoint is "converted to Int8" once at load
- * (abstract) -- int8mm_prepare_weight.
+ * as RTN); a 16- or 32-bit checkpoint is turned into int8 once, when it is
+ * loaded (abstract) -- int8mm_prepare_weight.
  *
  * What one int8mm_forward computes (X: M x K, W: K x N, both fp16 row-major):
  *   (a) O = ascending list of columns k with |X[m,k]| >= threshold for any m;
@@ -78,8 +78,8 @@ const char* int8mm_status_string(int8mm_status s);
 int int8mm_version(void);
 
 /* ------------------------------------------------------------------------ */
-/* Prepared (int8) weight -- "a 16/32-bit checkpoint can be loaded, converted */
-/* to Int8, and used immediately" (LLM.int8() abstract).                       */
+/* Prepared (int8) weight: the 16-bit checkpoint is converted to int8 once, at */
+/* load, and then used as it is (LLM.int8() page, abstract).                  */
 /* ------------------------------------------------------------------------ */
 
 /* Views into one caller-owned device buffer, filled by int8mm_prepare_weight.

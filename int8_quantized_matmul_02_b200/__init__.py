@@ -74,7 +74,7 @@ class PreparedWeight:
 
 
 def prepare_weight(W: torch.Tensor, keep_idx=(), stream=None) -> PreparedWeight:
-    """Convert a K x N fp16 CUDA weight to int8 once ("converted to Int8" at load)."""
+    """Convert a K x N fp16 CUDA weight to int8 once (at load, per the LLM.int8() abstract)."""
     lib = _abi.load()
     if not (W.is_cuda and W.dtype == torch.float16 and W.dim() == 2 and W.is_contiguous()):
         raise ValueError("W must be a contiguous 2-D float16 CUDA tensor (K x N)")

@@ -1,7 +1,7 @@
 // Decode-shaped LLM.int8() forward (M <= 16 rows of X) in one kernel.
 //
-// At small M the product is bound by reading the int8 weight once ("memory
-// loading is significantly more costly than computation", axolotl
+// At small M the product is bound by reading the int8 weight once: loading
+// weights from memory costs far more than the arithmetic on them (axolotl
 // "llama3-model-quantization", "Impact of Precision and Parameter Count on
 // Model Efficiency").  The kernel streams the weight through every CTA's TMA
 // ring from the moment the CTA starts and keeps the X-side steps that gate

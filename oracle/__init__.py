@@ -12,14 +12,13 @@ raw 16-bit patterns.  Each wrapper names the passage it follows:
 * outlier detection -- axolotl "llama3-model-quantization", "Understanding
   Outliers in Transformer Models": outliers sit in specific feature columns;
 * row / column quantisation -- "LLM.int8(): 8-bit Matrix Multiplication for
-  Transformers at Scale", abstract ("vector-wise quantization with separate
-  normalization constants for each inner product"), max normalisation from the
+  Transformers at Scale", abstract (vector-wise quantisation: every inner
+  product gets its own normalisation constants), max normalisation from the
   axolotl page's "Key Points", round-to-nearest from the nuQmm scite report;
-* 16-bit outlier product -- the same abstract ("mixed-precision
-  decomposition ... isolates the outlier feature dimensions into a 16-bit
-  matrix multiplication");
-* weight conversion once at load -- the same abstract ("loaded, converted to
-  Int8, and used immediately");
+* 16-bit outlier product -- the same abstract (the mixed-precision
+  decomposition moves the outlier feature dimensions into a matmul in 16 bit);
+* weight conversion once at load -- the same abstract (a 16-bit checkpoint is
+  turned into int8 when it is loaded and used from then on);
 * block-wise 8-bit codec -- the axolotl page's "8-Bit Optimizers" paragraphs
   (blocks normalised by their own maximum, an 8-bit index per value);
 * group-wise matmul -- the scite report for nuQmm (nuQmm / ZeroQuant use one

@@ -24,14 +24,34 @@ def _gpu(cuda_ok):
 
 
 def _run_case(M, K, N, n_seed, thr=6.0, path="auto", keep="seeded", cap=None, seed=0, mode="element",
-              lo=10.0, hi=60.0):
+              lo=10.0, hi=60.0, with_acc=True):
+    """One case against the oracle.  with_acc=False runs the kernels that
+    production calls run (no int32 debug output: the GEMM's instantiation
+    without the accumulator stores) and checks every intermediate it leaves
+    plus Y; with_acc=True also checks the int32 sums."""
     X, W, cols = synth.make_case(M, K, N, n_seed=n_seed, lo=lo, hi=hi, mode=mode, seed=seed)
     keep_idx = {"seeded": cols, "none": [], "all": list(range(K))}[keep]
     w = parity.gpu_prepare(W, keep_idx)
     prep, r = parity.oracle_full(X, W, keep_idx, thr)
     parity.check_weight(w, prep)
-    g = parity.gpu_forward(X, w, thr, path=path, cap=cap)
+    g = parity.gpu_forward(X, w, thr, path=path, cap=cap, with_acc=with_acc)
     return parity.check_forward_full(g, r), r
+
+
+def _both_instantiations(M, K, N, n_seed, path, seed, thr=6.0):
+    """The forward with and without the int32 debug output: each against the
+    oracle, and Y bit-identical between the two (the stores of the sums are
+    the only difference between the two kernels)."""
+    X, W, cols = synth.make_case(M, K, N, n_seed=n_seed, seed=seed)
+    w = parity.gpu_prepare(W, cols)
+    prep, r = parity.oracle_full(X, W, cols, thr)
+    g1 = parity.gpu_forward(X, w, thr, path=path, with_acc=True)
+    parity.check_forward_full(g1, r)
+    g0 = parity.gpu_forward(X, w, thr, path=path, with_acc=False)
+    parity.check_forward_full(g0, r)
+    assert torch.equal(g0["Y_dev"].view(torch.int16), g1["Y_dev"].view(torch.int16)), \
+        "Y differs between the kernels with and without the int32 output"
+    return r
 
 
 # ------------------------------------------------------------------ tiled GEMM path
@@ -44,9 +64,19 @@ def _run_case(M, K, N, n_seed, thr=6.0, path="auto", keep="seeded", cap=None, se
     (700, 1024, 1040, 5),     # several SM-pair tiles with a ragged pair
 ])
 @pytest.mark.parametrize("path", ["gemm", "gemm1sm"])
-def test_gemm_path_matches_oracle(M, K, N, n_seed, path):
-    """"gemm" uses SM-pair 256 x 256 tiles for M > 128; "gemm1sm" the single-SM kernel."""
-    _run_case(M, K, N, n_seed, path=path)
+@pytest.mark.parametrize("with_acc", [True, False])
+def test_gemm_path_matches_oracle(M, K, N, n_seed, path, with_acc):
+    """"gemm" uses SM-pair 256 x 256 tiles for M > 128; "gemm1sm" the single-SM
+    kernel.  with_acc=False is the instantiation every production call runs."""
+    _run_case(M, K, N, n_seed, path=path, with_acc=with_acc)
+
+
+@pytest.mark.parametrize("path", ["gemm", "gemm1sm", "decode"])
+@pytest.mark.parametrize("M,K,N,n_seed", [(8, 2048, 1040, 5), (300, 1040, 784, 4), (700, 1024, 1040, 65)])
+def test_production_kernels_match_debug_kernels(M, K, N, n_seed, path):
+    if path == "decode" and M > 16:
+        pytest.skip("the decode kernel takes M <= 16")
+    _both_instantiations(M, K, N, n_seed, path, seed=500 + M + n_seed)
 
 
 @pytest.mark.parametrize("M", [1, 8, 17, 64, 65, 129])
@@ -57,6 +87,13 @@ def test_gemm_path_row_counts(M):
 @pytest.mark.parametrize("n_seed", [0, 1, 15, 16, 17, 64, 65])
 def test_gemm_path_outlier_counts(n_seed):
     _, r = _run_case(160, 1024, 512, n_seed, path="gemm", seed=100 + n_seed)
+    assert r["idx"].size >= n_seed
+
+
+@pytest.mark.parametrize("n_seed", [0, 1, 64, 65])
+@pytest.mark.parametrize("path", ["gemm", "gemm1sm"])
+def test_gemm_path_outlier_counts_production_kernel(n_seed, path):
+    _, r = _run_case(300, 1024, 528, n_seed, path=path, seed=200 + n_seed, with_acc=False)
     assert r["idx"].size >= n_seed
 
 
@@ -99,8 +136,9 @@ def test_gemm_path_zero_rows_and_columns():
     (5, 128, 1040, 2),        # one full K block
     (16, 20480, 272, 7),      # the longest K the decode kernel takes (clusters of 8)
 ])
-def test_decode_path_matches_oracle(M, K, N, n_seed):
-    _run_case(M, K, N, n_seed, path="decode", seed=M * 31 + K)
+@pytest.mark.parametrize("with_acc", [True, False])
+def test_decode_path_matches_oracle(M, K, N, n_seed, with_acc):
+    _run_case(M, K, N, n_seed, path="decode", seed=M * 31 + K, with_acc=with_acc)
 
 
 @pytest.mark.parametrize("keep", ["none", "all"])
@@ -226,21 +264,34 @@ def test_wait_limit_reports_timeout_and_recovers(path):
 # ------------------------------------------------------------------ full-size workloads
 
 def _full_size(name, cap=1024, full_oracle=False):
+    """The workload at full size, in the launch configuration the benchmark
+    times (workspace capacity 1024 outlier columns), run twice: without the
+    int32 debug output (the kernels the benchmark runs) and with it.  Both
+    against the oracle; Y bit-identical between the two."""
     wl = synth.WORKLOADS[name]
     X, W, cols = synth.make_inputs(wl)
     w = parity.gpu_prepare(W, cols)
     prep = oracle.prepare_weight(W.numpy(), cols)
     parity.check_weight(w, prep)
+    del W
     cap = min(cap, wl.K)
-    g = parity.gpu_forward(X, w, wl.threshold, path="auto", cap=cap)
     if full_oracle:
         r = oracle.forward(X.numpy(), prep, wl.threshold)
-        parity.check_forward_full(g, r)
-        return r["idx"].size
-    steps = oracle.forward_steps_abc(X.numpy(), prep, wl.threshold)
-    pm, pn = synth.sample_points(wl.M, wl.N, 4096, seed=wl.seed, tiles=((128, 256), (128, 256)))
-    parity.check_forward_sampled(g, steps, prep, pm, pn)
-    return steps["idx"].size
+    else:
+        steps = oracle.forward_steps_abc(X.numpy(), prep, wl.threshold)
+        pm, pn = synth.sample_points(wl.M, wl.N, 4096, seed=wl.seed, tiles=((128, 256), (128, 256)))
+    ys = []
+    for with_acc in (False, True):
+        g = parity.gpu_forward(X, w, wl.threshold, path="auto", cap=cap, with_acc=with_acc)
+        if full_oracle:
+            parity.check_forward_full(g, r)
+        else:
+            parity.check_forward_sampled(g, steps, prep, pm, pn)
+        ys.append(g["Y_dev"])
+        del g
+    assert torch.equal(ys[0].view(torch.int16), ys[1].view(torch.int16)), \
+        "Y differs between the kernels with and without the int32 output"
+    return r["idx"].size if full_oracle else steps["idx"].size
 
 
 def test_full_size_decode():
@@ -248,7 +299,7 @@ def test_full_size_decode():
     assert n_o >= 6
 
 
-@pytest.mark.parametrize("name", ["prefill", "175b", "qkv_o123", "qkv_inf"])
+@pytest.mark.parametrize("name", ["prefill", "175b", "qkv_o0", "qkv_o12", "qkv_o48", "qkv_o123", "qkv_inf"])
 def test_full_size_sampled(name):
     n_o = _full_size(name)
     assert n_o >= synth.WORKLOADS[name].n_seed

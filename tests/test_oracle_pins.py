@@ -371,7 +371,7 @@ def test_points_match_full_forward():
 
 
 def test_eight_bit_share_on_decode_recipe():
-    """The abstract's "more than 99.9% of values are multiplied in 8-bit": with
+    """The abstract's claim that over 99.9 % of the values go through the 8-bit product: with
     the decode recipe's 6 seeded columns out of 4096 the share is 99.85%."""
     wl = synth.WORKLOADS["decode"]
     gen = __import__("torch").Generator().manual_seed(wl.seed)

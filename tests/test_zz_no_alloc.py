@@ -5,9 +5,10 @@ and output buffers from a host framework that owns all device memory, and
 latency-critical paths where cudaMalloc's cost and device-wide
 synchronisation are not acceptable.  int8mm_forward_decode_noalloc serves
 them with scratch memory in a fixed-size array inside the library.  This test
-calls it through the C-ABI and checks that it gives the same output as the
-regular entry point (int8mm_forward with a caller workspace), within the
-tolerance of the parity tests, on two calls in a row with different inputs.
+calls it through the C-ABI on two calls in a row with different inputs and
+checks each against the CPU oracle (within the tolerance of the parity tests)
+and against the regular entry point (int8mm_forward with a caller workspace,
+on the same kernel: bit-identical).
 
 This file is named so that pytest collects it last.
 """
@@ -19,6 +20,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import int8_quantized_matmul_02_b200 as i8
 from int8_quantized_matmul_02_b200 import _abi, synth
 from tests import parity
@@ -40,19 +42,29 @@ def _noalloc(lib, X: torch.Tensor, w: i8.PreparedWeight, thr: float) -> torch.Te
 
 @pytest.mark.parametrize("M,K,N,n_seed", [(8, 4096, 11008, 6), (16, 2048, 1040, 3), (1, 256, 384, 1)])
 def test_noalloc_matches_regular_entry_point_twice(cuda_ok, M, K, N, n_seed):
+    """Two calls in a row with different inputs.  Each call is checked against
+    the oracle (outlier count exact, Y within the parity tolerance) and against
+    int8mm_forward on the same fused decode kernel (Y bit-identical: only the
+    place of the scratch memory differs)."""
     lib = _abi.load()
     _, W, cols = synth.make_case(M, K, N, n_seed=n_seed, seed=7000 + M)
     w = i8.prepare_weight(W.cuda(), cols)
+    prep = oracle.prepare_weight(W.numpy(), cols)
     for call in range(2):  # the second call must not see the first call's scratch
         X, _, _ = synth.make_case(M, K, N, n_seed=n_seed, seed=7000 + M)
-        X = (X.float() * (1.0 + 0.25 * call)).half().cuda()
+        X = (X.float() * (1.0 + 0.25 * call)).half()
+        if call == 1:
+            X[:, (37 * M) % K] = 25.0  # one more outlier column on the second call
+        ref = oracle.forward(X.numpy(), prep, 6.0)
+        Xd = X.cuda()
         ws = i8.Workspace(M, K, N)
-        Y_ref = i8.forward(X, w, 6.0, workspace=ws)
+        Y_ref = i8.forward(Xd, w, 6.0, workspace=ws, path="decode")
         st_ref, n_ref = i8.device_status(ws)
         assert st_ref == 0
-        Y, n = _noalloc(lib, X, w, 6.0)
-        assert n == n_ref
-        parity.assert_y_close(Y.float().cpu().numpy(), Y_ref.float().cpu().numpy(), what=f"call {call}")
+        Y, n = _noalloc(lib, Xd, w, 6.0)
+        assert n == n_ref == ref["idx"].size
+        parity.assert_y_close(Y.float().cpu().numpy(), ref["y"].astype(np.float64), what=f"call {call} vs oracle")
+        assert torch.equal(Y.view(torch.int16), Y_ref.view(torch.int16)), f"call {call}: Y differs from int8mm_forward"
 
 
 def test_noalloc_rejects_sizes_beyond_its_limit(cuda_ok):
