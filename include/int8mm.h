@@ -183,6 +183,68 @@ int8mm_status int8mm_workspace_view_get(void* ws, size_t ws_bytes, int M, int K,
 int8mm_status int8mm_get_device_status(const void* ws, void* stream, int32_t* n_outliers);
 
 /* ------------------------------------------------------------------------ */
+/* Block-wise linear 8-bit codec (axolotl "llama3-model-quantization",      */
+/* "8-Bit Optimizers": blocks normalised by their own maximum, an 8-bit     */
+/* index per value).                                                         */
+/* ------------------------------------------------------------------------ */
+
+/* q (device, n int8) and absmax (device, ceil(n/B) fp32) of x (device, n
+ * fp32, finite): block b covers [b*B, min(n, (b+1)*B)), absmax[b] = max |x|
+ * over it, q = round_half_even(x * (127.0f / absmax[b])) (fp32 arithmetic;
+ * absmax 0 gives 0).  B % 4 == 0, B >= 4; x 16-byte, q and absmax 4-byte
+ * aligned. */
+int8mm_status int8mm_block_quantize(const float* x, int64_t n, int B, int8_t* q, float* absmax, void* stream);
+
+/* out (device, n fp32) = (q * absmax[block]) / 127 in fp32, the inverse of
+ * int8mm_block_quantize up to half a quantisation step.  out 16-byte
+ * aligned, q and absmax 4-byte aligned. */
+int8mm_status int8mm_block_dequantize(const int8_t* q, const float* absmax, int64_t n, int B, float* out,
+                                      void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* 4-bit weight-only product for decode-sized X ("4-Bit Inference" on the   */
+/* video page "8-bit Methods for Efficient Deep Learning with Tim Dettmers"; */
+/* axolotl "llama3-model-quantization", "Impact of Precision and Parameter  */
+/* Count on Model Efficiency": at small batch the weight bytes set the time). */
+/* ------------------------------------------------------------------------ */
+
+/* Views into one caller-owned device buffer, filled by
+ * int8mm_prepare_weight_int4.  codes: N rows of K/2 bytes; every 32-bit word
+ * holds 8 consecutive k of one output column as nibbles u = q + 8 (q in
+ * [-7, 7]) in the order k0 -> bits 0-3, k0+1 -> 16-19, k0+2 -> 4-7,
+ * k0+3 -> 20-23, k0+4 -> 8-11, k0+5 -> 24-27, k0+6 -> 12-15, k0+7 -> 28-31.
+ * absmax: N x (K/G) fp32, absmax[n*(K/G) + g] = max |W[k,n]| over the group
+ * g of G consecutive k. */
+typedef struct {
+    int32_t K, N, G;
+    uint8_t* codes;      /* device, N x K/2 bytes */
+    float* absmax;       /* device, N x K/G */
+} int8mm_int4_weight;
+
+/* Bytes of the buffer for a K x N weight with groups of G (0 when the shape
+ * breaks the rules: K, N >= 16, K % 128 == 0, N % 16 == 0, G % 128 == 0,
+ * G divides K, K <= 131072). */
+size_t int8mm_int4_weight_bytes(int K, int N, int G);
+
+/* Convert W (device, K x N fp16) to 4-bit codes once: per output column n and
+ * group g, absmax = max |W[k,n]|, q = round_half_even(W[k,n] * (7.0f /
+ * absmax)) (fp32) clamped to +-7, 0 when absmax is 0.  buf: 256-byte aligned
+ * device buffer of int8mm_int4_weight_bytes(K, N, G) bytes.  Stream-ordered;
+ * W must stay valid until the work on `stream` is done. */
+int8mm_status int8mm_prepare_weight_int4(const uint16_t* W, int K, int N, int G, void* buf, size_t buf_bytes,
+                                         int8mm_int4_weight* out, void* stream);
+
+/* Y (device, M x N fp16) = X (device, M x K fp16) times the 4-bit weight,
+ * 1 <= M <= 16:  y[m,n] = sum_k x[m,k] * (q[n,k] * absmax[n,g(k)] / 7), the
+ * products on the tensor cores with fp32 sums, rounded to fp16 once.
+ * status: device int32 word, zero before the call; a wait in the kernel that
+ * runs out sets bit 0 (INT8MM_ERR_TIMEOUT: outputs invalid).  Stream-ordered
+ * (programmatic dependent launch: the weight stream of a call starts while
+ * the previous kernel on the stream finishes). */
+int8mm_status int8mm_forward_int4(const uint16_t* X, int M, const int8mm_int4_weight* w, uint16_t* Y,
+                                  int32_t* status, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* Decode-sized forward that allocates nothing                               */
 /* ------------------------------------------------------------------------ */
 

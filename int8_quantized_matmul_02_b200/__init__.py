@@ -25,6 +25,8 @@ from ._abi import PATH_AUTO, PATH_DECODE, PATH_GEMM, PATH_GEMM_1SM, Int8mmError
 
 __all__ = [
     "PreparedWeight", "Workspace", "prepare_weight", "forward", "device_status", "library",
+    "block_quantize", "block_dequantize",
+    "Int4Weight", "prepare_weight_int4", "forward_int4", "unpack_int4_codes",
     "Int8mmError", "PATH_AUTO", "PATH_GEMM", "PATH_DECODE",
 ]
 
@@ -171,3 +173,109 @@ def device_status(workspace: Workspace, stream=None) -> tuple[int, int]:
         st = _abi.load().int8mm_get_device_status(ctypes.c_void_p(workspace.buf.data_ptr()), _stream(stream),
                                                   ctypes.byref(n))
     return int(st), int(n.value)
+
+
+# ---------------------------------------------------------------------------- block-wise 8-bit codec
+
+def block_quantize(x: torch.Tensor, B: int, q: torch.Tensor | None = None, absmax: torch.Tensor | None = None,
+                   stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Block-wise linear 8-bit codes of a float32 CUDA vector: block b covers
+    [b*B, min(n, (b+1)*B)) and is normalised by its own absolute maximum
+    (axolotl "llama3-model-quantization", "8-Bit Optimizers" paragraphs).
+    Returns (codes int8 of n, absmax float32 of ceil(n/B))."""
+    if not (x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()):
+        raise ValueError("x must be a contiguous float32 CUDA tensor")
+    n = x.numel()
+    nb = (n + B - 1) // B
+    q = torch.empty(n, dtype=torch.int8, device=x.device) if q is None else q
+    absmax = torch.empty(nb, dtype=torch.float32, device=x.device) if absmax is None else absmax
+    with torch.cuda.device(x.device):
+        _abi.check(_abi.load().int8mm_block_quantize(ctypes.c_void_p(x.data_ptr()), n, int(B),
+                                                     ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(absmax.data_ptr()),
+                                                     _stream(stream)), "int8mm_block_quantize")
+    return q, absmax
+
+
+def block_dequantize(q: torch.Tensor, absmax: torch.Tensor, B: int, out: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """float32 values (q * absmax[block]) / 127 of block-wise codes."""
+    if not (q.is_cuda and q.dtype == torch.int8 and q.is_contiguous()):
+        raise ValueError("q must be a contiguous int8 CUDA tensor")
+    n = q.numel()
+    out = torch.empty(n, dtype=torch.float32, device=q.device) if out is None else out
+    with torch.cuda.device(q.device):
+        _abi.check(_abi.load().int8mm_block_dequantize(ctypes.c_void_p(q.data_ptr()),
+                                                       ctypes.c_void_p(absmax.data_ptr()), n, int(B),
+                                                       ctypes.c_void_p(out.data_ptr()), _stream(stream)),
+                   "int8mm_block_dequantize")
+    return out
+
+
+# ---------------------------------------------------------------------------- 4-bit weight-only decode product
+
+class Int4Weight:
+    """A 4-bit weight in one device buffer (see ``int8mm_int4_weight``)."""
+
+    def __init__(self, buf: torch.Tensor, st: _abi.Int4Weight):
+        self.buf = buf
+        self.struct = st
+        self.K, self.N, self.G = st.K, st.N, st.G
+
+    @property
+    def codes(self) -> torch.Tensor:        # N x K/2 packed nibbles
+        return _view(self.buf, self.struct.codes, self.N * self.K // 2, torch.uint8, (self.N, self.K // 2))
+
+    @property
+    def absmax(self) -> torch.Tensor:       # N x K/G float32
+        return _view(self.buf, self.struct.absmax, self.N * (self.K // self.G), torch.float32,
+                      (self.N, self.K // self.G))
+
+
+def prepare_weight_int4(W: torch.Tensor, G: int, stream=None) -> Int4Weight:
+    """Convert a K x N fp16 CUDA weight to 4-bit codes with one constant per
+    output column and group of G consecutive k (once, at load)."""
+    lib = _abi.load()
+    if not (W.is_cuda and W.dtype == torch.float16 and W.dim() == 2 and W.is_contiguous()):
+        raise ValueError("W must be a contiguous 2-D float16 CUDA tensor (K x N)")
+    K, N = W.shape
+    nbytes = lib.int8mm_int4_weight_bytes(K, N, int(G))
+    if nbytes == 0:
+        raise Int8mmError(1, f"int8mm_int4_weight_bytes(K={K}, N={N}, G={G})")
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    st = _abi.Int4Weight()
+    with torch.cuda.device(W.device):
+        _abi.check(lib.int8mm_prepare_weight_int4(ctypes.c_void_p(W.data_ptr()), K, N, int(G),
+                                                  ctypes.c_void_p(buf.data_ptr()), nbytes, ctypes.byref(st),
+                                                  _stream(stream)), "int8mm_prepare_weight_int4")
+    return Int4Weight(buf, st)
+
+
+def forward_int4(X: torch.Tensor, w: Int4Weight, out: torch.Tensor | None = None,
+                 status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y = X W' with the 4-bit weight (X: M x K fp16 on the weight's device,
+    M <= 16).  ``status`` (int32 CUDA tensor of one zero word) receives
+    device-side errors; a fresh one is used when it is None."""
+    lib = _abi.load()
+    if X.dtype != torch.float16 or X.dim() != 2 or X.shape[1] != w.K or not X.is_cuda or not X.is_contiguous():
+        raise ValueError(f"X must be a contiguous float16 CUDA tensor of shape (M, {w.K})")
+    M = X.shape[0]
+    Y = out if out is not None else torch.empty(M, w.N, dtype=torch.float16, device=X.device)
+    status = status if status is not None else torch.zeros(1, dtype=torch.int32, device=X.device)
+    with torch.cuda.device(X.device):
+        _abi.check(lib.int8mm_forward_int4(ctypes.c_void_p(X.data_ptr()), M, ctypes.byref(w.struct),
+                                           ctypes.c_void_p(Y.data_ptr()), ctypes.c_void_p(status.data_ptr()),
+                                           _stream(stream)), "int8mm_forward_int4")
+    return Y
+
+
+def unpack_int4_codes(packed: np.ndarray) -> np.ndarray:
+    """Codes q (N x K int8) from the packed layout (N x K/2 uint8) that
+    ``int8mm_int4_weight`` documents; a layout helper, no arithmetic."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    N, half = packed.shape
+    words = packed.view("<u4").reshape(N, half // 4)
+    q = np.empty((N, half * 2), dtype=np.int8)
+    for i in range(8):
+        shift = (i & 1) * 16 + (i >> 1) * 4
+        q[:, i::8] = (((words >> shift) & 0xF).astype(np.int16) - 8).astype(np.int8)
+    return q

@@ -30,6 +30,8 @@ EXPORTS = (
     "int8mm_workspace_bytes", "int8mm_workspace_init", "int8mm_forward", "int8mm_forward_ex",
     "int8mm_workspace_view_get", "int8mm_get_device_status",
     "int8mm_forward_decode_noalloc", "int8mm_noalloc_device_status",
+    "int8mm_block_quantize", "int8mm_block_dequantize",
+    "int8mm_int4_weight_bytes", "int8mm_prepare_weight_int4", "int8mm_forward_int4",
 )
 
 
@@ -45,6 +47,11 @@ class Weight(ctypes.Structure):
         ("wq", ctypes.c_void_p), ("col_absmax", ctypes.c_void_p), ("w_keep", ctypes.c_void_p),
         ("keep_idx", ctypes.c_void_p), ("keep_slot", ctypes.c_void_p),
     ]
+
+
+class Int4Weight(ctypes.Structure):
+    _fields_ = [("K", ctypes.c_int32), ("N", ctypes.c_int32), ("G", ctypes.c_int32),
+                ("codes", ctypes.c_void_p), ("absmax", ctypes.c_void_p)]
 
 
 class ForwardOpts(ctypes.Structure):
@@ -101,6 +108,17 @@ def load(path: str | None = None):
     lib.int8mm_forward_decode_noalloc.restype = I
     lib.int8mm_noalloc_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
     lib.int8mm_noalloc_device_status.restype = I
+    L64 = ctypes.c_int64
+    lib.int8mm_block_quantize.argtypes = [P, L64, I, P, P, P]
+    lib.int8mm_block_quantize.restype = I
+    lib.int8mm_block_dequantize.argtypes = [P, P, L64, I, P, P]
+    lib.int8mm_block_dequantize.restype = I
+    lib.int8mm_int4_weight_bytes.argtypes = [I, I, I]
+    lib.int8mm_int4_weight_bytes.restype = S
+    lib.int8mm_prepare_weight_int4.argtypes = [P, I, I, I, P, S, ctypes.POINTER(Int4Weight), P]
+    lib.int8mm_prepare_weight_int4.restype = I
+    lib.int8mm_forward_int4.argtypes = [P, I, ctypes.POINTER(Int4Weight), P, P, P]
+    lib.int8mm_forward_int4.restype = I
     if path is None:
         _lib = lib
     return lib

@@ -13,9 +13,11 @@
 #include <vector>
 
 #include "int8mm.h"
+#include "codec_kernels.cuh"
 #include "decode_sm100.cuh"
 #include "gemm2sm_sm100.cuh"
 #include "gemm_sm100.cuh"
+#include "int4_sm100.cuh"
 #include "quant_kernels.cuh"
 
 namespace {
@@ -26,6 +28,9 @@ constexpr int kVersion = 100;  // 0.1.0
 constexpr uint64_t kDefaultWaitNs = 2000ull * 1000 * 1000;
 constexpr int kMaxK = 131072;
 constexpr int kMaxSmemOptin = 232448;  // 227 KB per block on sm_100
+// Two CTAs of 113 KB (plus the 1 KB the hardware keeps per CTA) fit in the
+// 228 KB of shared memory of one SM.
+constexpr int kDecSmallSmem = 113 * 1024;
 constexpr int kMaxDecodeRows = 16;
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -68,9 +73,15 @@ int8mm_status current_device(int* dev_out, DeviceInfo** info_out) {
                                  kGemmSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(k_gemm_int8_sm100<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGemmSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(k_decode_int8_sm100<8, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(k_decode_int8_sm100<8, 8, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kDecSmallSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(k_decode_int8_sm100<16, 16, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kDecSmallSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(k_decode_int8_sm100<8, 8, 384>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kMaxSmemOptin) != cudaSuccess ||
-            cudaFuncSetAttribute(k_decode_int8_sm100<16, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(k_decode_int8_sm100<16, 16, 384>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kMaxSmemOptin) != cudaSuccess ||
+            cudaFuncSetAttribute(k_int4_decode_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kMaxSmemOptin) != cudaSuccess ||
             cudaFuncSetAttribute(k_gemm_int8_2sm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kG2SmemBytes) != cudaSuccess ||
@@ -237,58 +248,58 @@ uint32_t fp16_threshold_bits2(float thr) {
     return lo | (lo << 16);
 }
 
-// Plan of the decode kernel: clusters of `cluster` CTAs split K (each CTA
-// one K range of the cluster's `tiles` 128-channel tiles), a TMA ring of
-// `stages` 16 KB boxes, and the shared-memory offsets.
+// Plan of the decode kernel: its shape (256 threads with at most
+// kDecSmallSmem bytes of shared memory, so that two CTAs fit on one SM, or
+// 384 threads with up to 227 KB), clusters of `cluster` CTAs splitting K, the
+// number of clusters (tiles shared out evenly, at most `cluster` per
+// cluster), a TMA ring of `stages` 16 KB boxes, and the shared-memory offsets.
 struct DecodePlan {
-    int cluster, tiles, stages, groups, grid, mr;  // mr: rows per chunk group (8 or 16)
-    uint32_t off_xq, off_mask, off_pre, off_list, off_xo, off_oslot, off_red, off_bars, bytes;
+    int threads, cluster, clusters, max_tiles, stages, groups, grid, mr;  // mr: rows per chunk group (8 or 16)
+    uint32_t tmem_cols;
+    uint32_t off_xq, off_mask, off_pre, off_xo, off_oslot, off_red, off_bars, bytes;
 };
 
-// False when (M, K, cap) does not fit the kernel: M > 16, a CTA's K range
-// wider than its X-side threads hold in registers, or shared memory.
-bool decode_plan(int M, int K, int N, int cap, int sms, DecodePlan* P) {
-    if (M < 1 || M > kMaxDecodeRows) return false;
+// (chunk, row) pairs each X-side thread holds in registers (template kP of
+// the kernel): rows per chunk group 8 -> 8 pairs, 16 -> 16 pairs.
+constexpr int decode_pairs(int mr) { return mr == 8 ? 8 : 16; }
+
+bool decode_plan_shape(int M, int K, int N, int sms, int threads, size_t smem_cap, int min_stages, DecodePlan* P) {
     const int kbt = cdiv(K, 128);
-    // a CTA's K range holds at most kDecPro 8-column chunks (kP * kDecPro / kR)
-    int cl = 0;
-    for (int c : {4, 8}) {
-        const int cc = std::min(c, kbt);
-        if (cdiv(kbt, cc) * 16 <= kDecPro) {
-            cl = cc;
-            break;
-        }
-    }
-    if (cl == 0) return false;
+    const int mr = M <= 8 ? 8 : 16;
+    const int chunks_max = decode_pairs(mr) * (threads - 64) / mr;  // 8-column chunks of X one CTA holds
     const int tiles = cdiv(N, kDecTileN);
-    // fewest tiles per cluster that keep the grid within one wave
-    int t = cl;
-    for (int c = 1; c <= cl; ++c) {
-        if ((long long)cl * cdiv(tiles, c) <= sms) {
-            t = c;
-            break;
-        }
-    }
     const int groups = (M + 7) / 8;
     const int nw = cdiv(K, 32);
-    const size_t xq = (size_t)(cdiv(kbt, cl) * groups + 1) * 1024;
-    const size_t mask = align_up((size_t)nw * 4, 16);
-    const size_t pre = align_up((size_t)nw * 4, 16);
-    const size_t list = align_up((size_t)std::min(K, std::max(cap, 1)) * 2, 16);
-    const size_t xo = (size_t)kDecSmemOutliers * 16 * 2;
-    const size_t oslot = (size_t)kDecSmemOutliers * 4;
-    const size_t red = (size_t)cl * kDecTileN * 8 * groups * 4;  // one partial-sum slot per CTA of the cluster
-    const size_t fixed = xq + mask + pre + list + xo + oslot + red;
-    for (int s = 16; s >= 4; --s) {
-        const size_t bars = (size_t)(2 * s + 5) * 8 + 256;
-        const size_t total = 1024 + (size_t)s * kDecStageBytes + fixed + bars;
-        if (total <= (size_t)kMaxSmemOptin) {
+    for (int c : {4, 8}) {
+        const int cl = std::min(c, kbt);
+        if (cdiv(kbt, cl) * 16 > chunks_max) continue;
+        // clusters: one CTA per SM when the tiles allow (at most cl tiles per
+        // cluster), else as many waves as needed with cl tiles per cluster
+        int ncl = std::max(1, std::min(tiles, sms / cl));
+        if (cdiv(tiles, ncl) > cl) ncl = cdiv(tiles, cl);
+        const int tmax = cdiv(tiles, ncl);
+        uint32_t tcols = 32;
+        while (tcols < (uint32_t)(32 * tmax)) tcols *= 2;
+        const size_t xq = (size_t)(cdiv(kbt, cl) * groups + 1) * 1024;
+        const size_t mask = align_up((size_t)nw * 4, 16);
+        const size_t pre = align_up((size_t)nw * 4, 16);
+        const size_t xo = (size_t)kDecSmemOutliers * 16 * 2;
+        const size_t oslot = (size_t)kDecSmemOutliers * 4;
+        const size_t red = (size_t)(cl - 1) * kDecTileN * 8 * groups * 4;  // one partial-sum slot per peer
+        const size_t fixed = xq + mask + pre + xo + oslot + red;
+        for (int s = 16; s >= min_stages; --s) {
+            const size_t bars = (size_t)(2 * s + kDecMaxTiles + 4) * 8 + 256;  // + TMEM address, abort flag, row maxima, count, scales
+            const size_t total = 1024 + (size_t)s * kDecStageBytes + fixed + bars;
+            if (total > smem_cap) continue;
+            P->threads = threads;
             P->cluster = cl;
-            P->tiles = t;
+            P->clusters = ncl;
+            P->max_tiles = tmax;
             P->stages = s;
             P->groups = groups;
-            P->grid = cl * cdiv(tiles, t);
-            P->mr = M <= 8 ? 8 : 16;
+            P->grid = cl * ncl;
+            P->mr = mr;
+            P->tmem_cols = tcols;
             size_t o = (size_t)s * kDecStageBytes;
             P->off_xq = (uint32_t)o;
             o += xq;
@@ -296,8 +307,6 @@ bool decode_plan(int M, int K, int N, int cap, int sms, DecodePlan* P) {
             o += mask;
             P->off_pre = (uint32_t)o;
             o += pre;
-            P->off_list = (uint32_t)o;
-            o += list;
             P->off_xo = (uint32_t)o;
             o += xo;
             P->off_oslot = (uint32_t)o;
@@ -310,6 +319,14 @@ bool decode_plan(int M, int K, int N, int cap, int sms, DecodePlan* P) {
         }
     }
     return false;
+}
+
+// False when (M, K) does not fit the kernel: M > 16, or a CTA's K range wider
+// than its X-side threads hold in registers even in clusters of 8.
+bool decode_plan(int M, int K, int N, int sms, DecodePlan* P) {
+    if (M < 1 || M > kMaxDecodeRows) return false;
+    return decode_plan_shape(M, K, N, sms, 256, kDecSmallSmem, 4, P) ||
+           decode_plan_shape(M, K, N, sms, 384, kMaxSmemOptin, 4, P);
 }
 
 // Parameters of one decode launch (the workspace pointers are the caller's).
@@ -329,14 +346,14 @@ DecodeParams decode_params(const uint16_t* X, int M, const int8mm_weight* w, flo
     p.Y = Y;
     p.num_tiles = cdiv(w->N, kDecTileN);
     p.kb_total = cdiv(w->K, 128);
+    p.num_clusters = dp.clusters;
     p.cluster = dp.cluster;
-    p.tiles_per_cluster = dp.tiles;
     p.stages = dp.stages;
     p.groups = dp.groups;
+    p.tmem_cols = dp.tmem_cols;
     p.off_xq = dp.off_xq;
     p.off_mask = dp.off_mask;
     p.off_pre = dp.off_pre;
-    p.off_list = dp.off_list;
     p.off_xo = dp.off_xo;
     p.off_oslot = dp.off_oslot;
     p.off_red = dp.off_red;
@@ -346,9 +363,81 @@ DecodeParams decode_params(const uint16_t* X, int M, const int8mm_weight* w, flo
 
 cudaError_t launch_decode(const DecodePlan& dp, const CUtensorMap& tm_w, const DecodeParams& p, cudaStream_t s,
                           bool pdl) {
+    const dim3 grid(dp.grid), block(dp.threads);
+    if (dp.threads == 256) {
+        if (dp.mr == 8)
+            return launch_ex(k_decode_int8_sm100<8, decode_pairs(8), 256>, grid, block, dp.bytes, s, pdl, dp.cluster, tm_w, p);
+        return launch_ex(k_decode_int8_sm100<16, decode_pairs(16), 256>, grid, block, dp.bytes, s, pdl, dp.cluster, tm_w, p);
+    }
     if (dp.mr == 8)
-        return launch_ex(k_decode_int8_sm100<8, 8>, dim3(dp.grid), dim3(kDecThreads), dp.bytes, s, pdl, dp.cluster, tm_w, p);
-    return launch_ex(k_decode_int8_sm100<16, 16>, dim3(dp.grid), dim3(kDecThreads), dp.bytes, s, pdl, dp.cluster, tm_w, p);
+        return launch_ex(k_decode_int8_sm100<8, decode_pairs(8), 384>, grid, block, dp.bytes, s, pdl, dp.cluster, tm_w, p);
+    return launch_ex(k_decode_int8_sm100<16, decode_pairs(16), 384>, grid, block, dp.bytes, s, pdl, dp.cluster, tm_w, p);
+}
+
+// ------------------------------------------------------------------ 4-bit weight-only decode
+
+constexpr int kInt4MaxRows = 16;
+
+struct Int4Layout {
+    size_t codes, absmax, total;
+};
+
+Int4Layout int4_layout(int K, int N, int G) {
+    Int4Layout L{};
+    L.codes = 0;
+    size_t o = align_up((size_t)N * (K / 2), 256);
+    L.absmax = o;
+    o = align_up(o + (size_t)N * (K / G) * 4, 256);
+    L.total = o;
+    return L;
+}
+
+bool int4_shape_ok(int K, int N, int G) {
+    return K >= 128 && N >= 16 && K % 128 == 0 && N % 16 == 0 && K <= kMaxK && G >= 128 && G % 128 == 0 && K % G == 0;
+}
+
+// Plan of the 4-bit kernel: clusters of `cluster` CTAs split K in 256-k
+// boxes, tiles shared out as in the 8-bit decode plan; two CTAs per SM when
+// the plan fits in kDecSmallSmem.
+struct Int4Plan {
+    int cluster, clusters, stages, xrows, grid;
+    uint32_t tmem_cols, off_x, off_red, off_bars, bytes;
+};
+
+bool int4_plan(int M, int K, int N, int sms, Int4Plan* P) {
+    if (M < 1 || M > kInt4MaxRows) return false;
+    const int kbt = cdiv(K, kI4BoxK);
+    const int tiles = cdiv(N, kI4TileN);
+    const int xrows = M <= 8 ? 8 : 16;
+    for (size_t cap : {(size_t)kDecSmallSmem, (size_t)kMaxSmemOptin}) {
+        for (int c : {4, 8}) {
+            const int cl = std::min(c, kbt);
+            int ncl = std::max(1, std::min(tiles, sms / cl));
+            if (cdiv(tiles, ncl) > cl) ncl = cdiv(tiles, cl);
+            const size_t xb = (size_t)cdiv(kbt, cl) * (kI4BoxK / 64) * xrows * 128 + 1024;  // + the row-8 overhang
+            const size_t red = (size_t)(cl - 1) * kI4TileN * xrows * 4;
+            for (int s = 12; s >= 3; --s) {
+                const size_t bars = (size_t)(2 * s + 4 + 2 * kI4DSlots + 3) * 8 + 64;
+                const size_t total = 1024 + (size_t)s * kI4StageBytes + xb + red + bars;
+                if (total > cap) continue;
+                P->cluster = cl;
+                P->clusters = ncl;
+                P->stages = s;
+                P->xrows = xrows;
+                P->grid = cl * ncl;
+                P->tmem_cols = 256;
+                size_t o = (size_t)s * kI4StageBytes;
+                P->off_x = (uint32_t)o;
+                o += xb;
+                P->off_red = (uint32_t)o;
+                o += red;
+                P->off_bars = (uint32_t)align_up(o, 8);
+                P->bytes = (uint32_t)total;
+                return true;
+            }
+        }
+    }
+    return false;
 }
 
 // ------------------------------------------------------------------ no-allocation decode forward
@@ -544,7 +633,7 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
 
     // whether the decode kernel fits does not depend on the device; its grid does
     DecodePlan dp{};
-    const bool decode_fits = decode_plan(M, K, N, max_outliers, 1 << 20, &dp);
+    const bool decode_fits = decode_plan(M, K, N, 1 << 20, &dp);
     bool use_decode;
     if (path == INT8MM_PATH_DECODE) {
         if (!decode_fits) return INT8MM_ERR_INVALID_ARGUMENT;
@@ -558,7 +647,7 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
     DeviceInfo* info;
     int8mm_status st = current_device(&dev, &info);
     if (st != INT8MM_OK) return st;
-    if (use_decode && !decode_plan(M, K, N, max_outliers, info->sm_count, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (use_decode && !decode_plan(M, K, N, info->sm_count, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* b = static_cast<uint8_t*>(ws);
@@ -703,13 +792,13 @@ int8mm_status int8mm_forward_decode_noalloc(const uint16_t* X, int M, const int8
     const NoAllocLayout L = noalloc_layout(M, K);
     if (L.total > kNoAllocBytes) return INT8MM_ERR_INVALID_ARGUMENT;
     DecodePlan dp{};
-    if (!decode_plan(M, K, N, cap, 1 << 20, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!decode_plan(M, K, N, 1 << 20, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
 
     int dev;
     DeviceInfo* info;
     int8mm_status st = current_device(&dev, &info);
     if (st != INT8MM_OK) return st;
-    if (!decode_plan(M, K, N, cap, info->sm_count, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!decode_plan(M, K, N, info->sm_count, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
     uint8_t* b = nullptr;
     st = noalloc_scratch(dev, &b);
     if (st != INT8MM_OK) return st;
@@ -741,6 +830,115 @@ int8mm_status int8mm_noalloc_device_status(void* stream, int32_t* n_outliers) {
     st = noalloc_scratch(dev, &b);
     if (st != INT8MM_OK) return st;
     return int8mm_get_device_status(b, stream, n_outliers);
+}
+
+int8mm_status int8mm_block_quantize(const float* x, int64_t n, int B, int8_t* q, float* absmax, void* stream) {
+    if (!x || !q || !absmax || n < 1 || B < 4 || B % 4 != 0) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!aligned(x, 16) || !aligned(q, 4) || !aligned(absmax, 4)) return INT8MM_ERR_MISALIGNED;
+    int dev;
+    DeviceInfo* info;
+    int8mm_status st = current_device(&dev, &info);
+    if (st != INT8MM_OK) return st;
+    const long long nblocks = (n + B - 1) / B;
+    const int grid = (int)std::max<long long>(1, std::min<long long>((nblocks + 7) / 8, (long long)info->sm_count * 16));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int kv = (B + 127) / 128;  // float4 chunks per lane for the whole block
+    cudaError_t e;
+    if (kv <= 1) e = launch(k_block_quant<1>, dim3(grid), dim3(256), 0, s, false, x, (long long)n, B, nblocks, q, absmax);
+    else if (kv <= 2) e = launch(k_block_quant<2>, dim3(grid), dim3(256), 0, s, false, x, (long long)n, B, nblocks, q, absmax);
+    else if (kv <= 4) e = launch(k_block_quant<4>, dim3(grid), dim3(256), 0, s, false, x, (long long)n, B, nblocks, q, absmax);
+    else if (kv <= 8) e = launch(k_block_quant<8>, dim3(grid), dim3(256), 0, s, false, x, (long long)n, B, nblocks, q, absmax);
+    else if (kv <= 16) e = launch(k_block_quant<16>, dim3(grid), dim3(256), 0, s, false, x, (long long)n, B, nblocks, q, absmax);
+    else e = launch(k_block_quant<0>, dim3(grid), dim3(256), 0, s, false, x, (long long)n, B, nblocks, q, absmax);
+    return cuda_status(e);
+}
+
+int8mm_status int8mm_block_dequantize(const int8_t* q, const float* absmax, int64_t n, int B, float* out,
+                                      void* stream) {
+    if (!q || !absmax || !out || n < 1 || B < 4 || B % 4 != 0) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!aligned(q, 4) || !aligned(absmax, 4) || !aligned(out, 16)) return INT8MM_ERR_MISALIGNED;
+    int dev;
+    DeviceInfo* info;
+    int8mm_status st = current_device(&dev, &info);
+    if (st != INT8MM_OK) return st;
+    const long long nq = (n + 3) / 4;
+    const int grid = (int)std::max<long long>(1, std::min<long long>((nq + 255) / 256, (long long)info->sm_count * 16));
+    return cuda_status(launch(k_block_dequant, dim3(grid), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream), false,
+                              q, absmax, (long long)n, B, out));
+}
+
+size_t int8mm_int4_weight_bytes(int K, int N, int G) {
+    if (!int4_shape_ok(K, N, G)) return 0;
+    return int4_layout(K, N, G).total;
+}
+
+int8mm_status int8mm_prepare_weight_int4(const uint16_t* W, int K, int N, int G, void* buf, size_t buf_bytes,
+                                         int8mm_int4_weight* out, void* stream) {
+    if (!W || !buf || !out || !int4_shape_ok(K, N, G)) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!aligned(W, 16) || !aligned(buf, 256)) return INT8MM_ERR_MISALIGNED;
+    const Int4Layout L = int4_layout(K, N, G);
+    if (buf_bytes < L.total) return INT8MM_ERR_WORKSPACE_TOO_SMALL;
+    int dev;
+    DeviceInfo* info;
+    int8mm_status st = current_device(&dev, &info);
+    if (st != INT8MM_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* b = static_cast<uint8_t*>(buf);
+    int8mm_int4_weight w{};
+    w.K = K;
+    w.N = N;
+    w.G = G;
+    w.codes = b + L.codes;
+    w.absmax = reinterpret_cast<float*>(b + L.absmax);
+    const long long na = (long long)(K / G) * N, nc = (long long)(K / 8) * N;
+    cudaError_t e = launch(k_int4_absmax, dim3((unsigned)cdiv(na, 256)), dim3(256), 0, s, false, W, K, N, G, w.absmax);
+    if (e == cudaSuccess)
+        e = launch(k_int4_pack, dim3((unsigned)cdiv(nc, 256)), dim3(256), 0, s, false, W, K, N, G,
+                   (const float*)w.absmax, reinterpret_cast<uint32_t*>(w.codes));
+    if (e != cudaSuccess) return cuda_status(e);
+    *out = w;
+    return INT8MM_OK;
+}
+
+int8mm_status int8mm_forward_int4(const uint16_t* X, int M, const int8mm_int4_weight* w, uint16_t* Y,
+                                  int32_t* status, void* stream) {
+    if (!X || !w || !Y || !status || !w->codes || !w->absmax) return INT8MM_ERR_INVALID_ARGUMENT;
+    const int K = w->K, N = w->N;
+    if (!int4_shape_ok(K, N, w->G) || M < 1 || M > kInt4MaxRows) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(w->codes, 256) || !aligned(status, 4))
+        return INT8MM_ERR_MISALIGNED;
+    int dev;
+    DeviceInfo* info;
+    int8mm_status st = current_device(&dev, &info);
+    if (st != INT8MM_OK) return st;
+    Int4Plan pl{};
+    if (!int4_plan(M, K, N, info->sm_count, &pl)) return INT8MM_ERR_INVALID_ARGUMENT;
+    CUtensorMap tm_w, tm_x;
+    if (!make_map(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)K / 2, N, (uint64_t)K / 2, 128, kI4TileN) ||
+        !make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, K, M, (uint64_t)K * 2, 64, pl.xrows))
+        return INT8MM_ERR_CUDA;
+    Int4Params p{};
+    p.absmax = w->absmax;
+    p.Y = Y;
+    p.status = status;
+    p.wait_limit_ns = kDefaultWaitNs;
+    p.test_flags = 0;
+    p.M = M;
+    p.K = K;
+    p.N = N;
+    p.G = w->G;
+    p.num_tiles = cdiv(N, kI4TileN);
+    p.kb_total = cdiv(K, kI4BoxK);
+    p.num_clusters = pl.clusters;
+    p.cluster = pl.cluster;
+    p.stages = pl.stages;
+    p.xrows = pl.xrows;
+    p.tmem_cols = pl.tmem_cols;
+    p.off_x = pl.off_x;
+    p.off_red = pl.off_red;
+    p.off_bars = pl.off_bars;
+    return cuda_status(launch_ex(k_int4_decode_sm100, dim3(pl.grid), dim3(kI4Threads), pl.bytes,
+                                 reinterpret_cast<cudaStream_t>(stream), true, pl.cluster, tm_w, tm_x, p));
 }
 
 }  // extern "C"

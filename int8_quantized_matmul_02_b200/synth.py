@@ -126,3 +126,29 @@ def sample_points(M: int, N: int, count: int, seed: int, tiles=((128, 256),)):
     pm.append(np.array([M - 1, M - 1, 0]))
     pn.append(np.array([N - 1, 0, N - 1]))
     return np.concatenate(pm).astype(np.int32), np.concatenate(pn).astype(np.int32)
+
+
+# ----------------------------------------------------------------------------- variants of the path
+
+# The 4-bit weight-only product runs on the decode workload's X and W; its
+# group size is the one the scite report for nuQmm quotes from GPTQ (1024),
+# with 128 as the finer setting.
+INT4_GROUPS = (1024, 128)
+
+# Block-wise codec workload: the fp32 state of one weight of the 175B-scale FFN
+# (4096 x 12288 values), blocks of 2048.
+CODEC_N = 4096 * 12288
+CODEC_BLOCK = 2048
+CODEC_SEED = 5000
+
+
+def make_codec_vector(n: int = CODEC_N, seed: int = CODEC_SEED) -> torch.Tensor:
+    """A heavy-tailed fp32 vector, N(0,1) * exp(N(0,1)), with 0.1 % of the
+    values multiplied by 50: an optimizer state whose outliers would waste the
+    bits of a single global constant (axolotl "llama3-model-quantization",
+    "8-Bit Optimizers" paragraphs)."""
+    gen = torch.Generator().manual_seed(seed)
+    x = torch.randn(n, generator=gen) * torch.exp(torch.randn(n, generator=gen))
+    pick = torch.rand(n, generator=gen) < 0.001
+    x[pick] *= 50.0
+    return x.contiguous()

@@ -134,7 +134,10 @@ def test_gemm_path_zero_rows_and_columns():
     (3, 2048, 11008, 1),
     (4, 16, 272, 1),          # one 16-column K block: a cluster of one CTA
     (5, 128, 1040, 2),        # one full K block
-    (16, 20480, 272, 7),      # the longest K the decode kernel takes (clusters of 8)
+    (16, 20480, 272, 7),      # the longest K the decode kernel takes (clusters of 8, one CTA per SM)
+    (8, 11008, 4096, 6),      # FFN down-projection shape: clusters of 8, two CTAs per SM, 2-3 tiles each
+    (8, 16384, 1040, 5),      # M <= 8 on the one-CTA-per-SM shape
+    (16, 12288, 2048, 4),     # M > 8 on the one-CTA-per-SM shape, clusters of 8
 ])
 @pytest.mark.parametrize("with_acc", [True, False])
 def test_decode_path_matches_oracle(M, K, N, n_seed, with_acc):
