@@ -438,6 +438,51 @@ def run_codec(steps: int, warmup: int, dev):
             "quant_bytes": 4.0 * n + n + 4.0 * nb, "dequant_bytes": 1.0 * n + 4.0 * nb + 4.0 * n}
 
 
+def run_grouped(wl, G: int, steps: int, warmup: int, dev, cap: int):
+    """Group-wise forward (one constant per row/column and group of G
+    consecutive k) on a large-M workload; the SM-pair GEMM kernel timed by
+    events the library records around it."""
+    import ctypes
+
+    import int8_quantized_matmul_02_b200 as i8
+    from int8_quantized_matmul_02_b200 import _abi
+
+    X, W, cols = synth.make_inputs(wl)
+    Xd = X.to(dev)
+    w = i8.prepare_weight_grouped(W.to(dev), G, cols)
+    del W
+    ws = i8.Workspace(wl.M, wl.K, wl.N, cap, device=dev, G=G)
+    Y = torch.empty(wl.M, wl.N, dtype=torch.float16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    lib = i8.library()
+    evs = event_pairs(steps, stream)
+
+    def step(ev=None):
+        opts = _abi.ForwardOpts(0, None, 0, ctypes.c_void_p(ev[0].cuda_event) if ev else None,
+                                ctypes.c_void_p(ev[1].cuda_event) if ev else None)
+        _abi.check(lib.int8mm_forward_grouped(ctypes.c_void_p(Xd.data_ptr()), wl.M, ctypes.byref(w.struct),
+                                              float(wl.threshold), ws.max_outliers, ctypes.c_void_p(Y.data_ptr()),
+                                              ctypes.c_void_p(ws.buf.data_ptr()), ws.nbytes, ctypes.byref(opts),
+                                              ctypes.c_void_p(stream.cuda_stream)), "int8mm_forward_grouped")
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        a.record(stream)
+        for i in range(steps):
+            step(evs[i])
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+    st, n_o = i8.device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"grouped device status {st}")
+    return {"total_ms": a.elapsed_time(b), "kern_ms": [x.elapsed_time(y) for x, y in evs], "n_o": n_o,
+            "clocks": clk.summary()}
+
+
 _pg = None
 
 
@@ -697,6 +742,32 @@ def main():
                 line["gpu_launches"] += 2 * args.steps
             except Exception as exc:
                 line["block_codec"] = {"error": f"{type(exc).__name__}: {exc}"}
+        if not args.no_variants:
+            line["grouped"] = {}
+            for G in synth.GROUP_SIZES:
+                try:
+                    rg = run_grouped(wl, G, args.steps, args.warmup, dev, cap)
+                except Exception as exc:
+                    line["grouped"][f"G{G}"] = {"error": f"{type(exc).__name__}: {exc}"}
+                    continue
+                step_s = rg["total_ms"] * 1e-3 / args.steps
+                k_s = statistics.mean(rg["kern_ms"]) * 1e-3
+                sus = rg["total_ms"] * 1e-3 >= 2.0
+                pk8 = (pk["bf16_tflops_sustained"] if sus else pk["bf16_tflops"]) * INT8_PER_BF16
+                line["grouped"][f"G{G}"] = {
+                    "workload": "group-wise variant, %s, groups of %d" % (WORKLOAD_NAMES[args.workload], G),
+                    "metric": "int8-decomposed matmul TOPS", "unit": "TOPS", "value": wl.ops / step_s / 1e12,
+                    "ms_per_step": step_s * 1e3, "frac_of_nominal_int8": wl.ops / step_s / 1e12 / NOMINAL_INT8_TOPS,
+                    "outlier_columns_detected": rg["n_o"],
+                    "roofline": {"bound": "tensor", "kernel": "k_gemm_int8_grouped", "achieved": wl.ops / k_s / 1e12,
+                                 "peak": pk8, "unit": "TFLOP/s", "frac": wl.ops / k_s / 1e12 / pk8,
+                                 "ms_per_launch": k_s * 1e3,
+                                 "peak_note": "dense int8 = 2 x %s bf16 (%s) cuBLAS peak"
+                                              % (pk_kind, "sustained" if sus else "burst")},
+                    "clocks": rg["clocks"],
+                }
+                line["gpu_launches"] += 4 * args.steps
+                torch.cuda.empty_cache()
         if not args.no_configs:
             line["configs"] = {}
             for name in ("prefill", "qkv_o0", "qkv_o12", "qkv_o48", "qkv_o123", "qkv_inf"):

@@ -202,6 +202,58 @@ int8mm_status int8mm_block_dequantize(const int8_t* q, const float* absmax, int6
                                       void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Group-wise variant: one normalisation constant per row of X and group of */
+/* G consecutive k, and per output column and group (the granularity of     */
+/* nuQmm and ZeroQuant, finer than vector-wise: scite report for nuQmm,     */
+/* citing snippets).  The outlier decomposition is unchanged.              */
+/* ------------------------------------------------------------------------ */
+
+/* As int8mm_weight, with col_absmax holding (K/G) x N constants:
+ * col_absmax[g*N + n] = max |W[k,n]| over the group g of G consecutive k, and
+ * Wq[n,k] quantised with the constant of its group. */
+typedef struct {
+    int32_t K, N, G, n_keep;
+    int8_t* wq;          /* device, N x K int8 */
+    float* col_absmax;   /* device, (K/G) x N */
+    uint16_t* w_keep;    /* device, n_keep x N fp16 */
+    int32_t* keep_idx;   /* device, n_keep */
+    int32_t* keep_slot;  /* device, K */
+} int8mm_grouped_weight;
+
+/* Bytes of the weight buffer (0 when a rule is broken: the int8mm_weight
+ * rules, plus G a multiple of 128 that divides K). */
+size_t int8mm_grouped_weight_bytes(int K, int N, int G, int n_keep);
+
+/* As int8mm_prepare_weight, with one constant per column and group. */
+int8mm_status int8mm_prepare_weight_grouped(const uint16_t* W, int K, int N, int G, const int32_t* keep_idx_host,
+                                            int n_keep, void* buf, size_t buf_bytes, int8mm_grouped_weight* out,
+                                            void* stream);
+
+/* Bytes of the workspace of a group-wise forward (its row constants are
+ * M x K/G). */
+size_t int8mm_grouped_workspace_bytes(int M, int K, int N, int G, int max_outliers);
+
+/* Views into a group-wise workspace; row_absmax holds M x (K/G) constants,
+ * row_absmax[m*(K/G) + g]. */
+int8mm_status int8mm_grouped_workspace_view_get(void* ws, size_t ws_bytes, int M, int K, int N, int G,
+                                                int max_outliers, int8mm_workspace_view* out);
+
+/* Y = X W by the group-wise method, any M >= 1:
+ *   ra[m,g] = max |X[m,k]| over the non-outlier k of group g, codes with the
+ *   group's scale RN32(127/ra[m,g]) (half-even, outlier columns 0),
+ *   acc_g = exact int32 sum over the group, and
+ *   y = fp16( sum_g ((float(acc_g) * ra[m,g]) * ca[g,n]) / 16129  (fp32, ascending g)
+ *             + sum_j X[m,O[j]] * Wo[j,n] ),
+ * where a non-kept outlier row is dequantised with its own group's constant.
+ * opts: path is ignored (SM-pair tcgen05 kernel); acc_out, if set, receives
+ * the per-group int32 sums, M x N x (K/G), acc_out[(m*N + n)*(K/G) + g];
+ * events, wait limit and test flags as for int8mm_forward_ex.  Device-side
+ * errors are read with int8mm_get_device_status. */
+int8mm_status int8mm_forward_grouped(const uint16_t* X, int M, const int8mm_grouped_weight* w, float threshold,
+                                     int max_outliers, uint16_t* Y, void* ws, size_t ws_bytes,
+                                     const int8mm_forward_opts* opts, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* 4-bit weight-only product for decode-sized X ("4-Bit Inference" on the   */
 /* video page "8-bit Methods for Efficient Deep Learning with Tim Dettmers"; */
 /* axolotl "llama3-model-quantization", "Impact of Precision and Parameter  */

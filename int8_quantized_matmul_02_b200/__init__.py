@@ -27,6 +27,7 @@ __all__ = [
     "PreparedWeight", "Workspace", "prepare_weight", "forward", "device_status", "library",
     "block_quantize", "block_dequantize",
     "Int4Weight", "prepare_weight_int4", "forward_int4", "unpack_int4_codes",
+    "GroupedWeight", "prepare_weight_grouped", "forward_grouped",
     "Int8mmError", "PATH_AUTO", "PATH_GEMM", "PATH_DECODE",
 ]
 
@@ -98,13 +99,17 @@ def prepare_weight(W: torch.Tensor, keep_idx=(), stream=None) -> PreparedWeight:
 class Workspace:
     """Device scratch of one forward shape; zero-filled at creation."""
 
-    def __init__(self, M: int, K: int, N: int, max_outliers: int | None = None, device=None):
+    def __init__(self, M: int, K: int, N: int, max_outliers: int | None = None, device=None, G: int | None = None):
+        """G: group size of a group-wise forward (None: vector-wise)."""
         lib = _abi.load()
-        self.M, self.K, self.N = M, K, N
+        self.M, self.K, self.N, self.G = M, K, N, G
         self.max_outliers = K if max_outliers is None else int(max_outliers)
-        self.nbytes = lib.int8mm_workspace_bytes(M, K, N, self.max_outliers)
+        if G is None:
+            self.nbytes = lib.int8mm_workspace_bytes(M, K, N, self.max_outliers)
+        else:
+            self.nbytes = lib.int8mm_grouped_workspace_bytes(M, K, N, int(G), self.max_outliers)
         if self.nbytes == 0:
-            raise Int8mmError(1, f"int8mm_workspace_bytes(M={M}, K={K}, N={N}, max_outliers={self.max_outliers})")
+            raise Int8mmError(1, f"workspace bytes (M={M}, K={K}, N={N}, max_outliers={self.max_outliers}, G={G})")
         self.buf = torch.zeros(self.nbytes, dtype=torch.uint8, device=device or "cuda")
 
     def reset(self, stream=None) -> None:
@@ -116,15 +121,23 @@ class Workspace:
     def view(self) -> dict:
         """Torch views of the intermediates the last forward left in the workspace."""
         v = _abi.WorkspaceView()
-        _abi.check(_abi.load().int8mm_workspace_view_get(ctypes.c_void_p(self.buf.data_ptr()), self.nbytes, self.M,
-                                                         self.K, self.N, self.max_outliers, ctypes.byref(v)),
-                   "int8mm_workspace_view_get")
+        lib = _abi.load()
+        if self.G is None:
+            _abi.check(lib.int8mm_workspace_view_get(ctypes.c_void_p(self.buf.data_ptr()), self.nbytes, self.M,
+                                                     self.K, self.N, self.max_outliers, ctypes.byref(v)),
+                       "int8mm_workspace_view_get")
+        else:
+            _abi.check(lib.int8mm_grouped_workspace_view_get(ctypes.c_void_p(self.buf.data_ptr()), self.nbytes, self.M,
+                                                             self.K, self.N, int(self.G), self.max_outliers,
+                                                             ctypes.byref(v)), "int8mm_grouped_workspace_view_get")
+        nr = 1 if self.G is None else self.K // self.G
         b = self.buf
         return {
             "status": _view(b, v.status, 1, torch.int32),
             "n_outliers": _view(b, v.n_outliers, 1, torch.int32),
             "outlier_idx": _view(b, v.outlier_idx, self.K, torch.int32),
-            "row_absmax": _view(b, v.row_absmax, self.M, torch.float32),
+            "row_absmax": (_view(b, v.row_absmax, self.M, torch.float32) if self.G is None else
+                           _view(b, v.row_absmax, self.M * nr, torch.float32, (self.M, nr))),
             "xq": _view(b, v.xq, self.M * self.K, torch.int8, (self.M, self.K)),
             "xo": _view(b, v.xo, self.M * v.kp, torch.float16, (self.M, v.kp)) if v.kp else None,
             "kp": v.kp,
@@ -279,3 +292,77 @@ def unpack_int4_codes(packed: np.ndarray) -> np.ndarray:
         shift = (i & 1) * 16 + (i >> 1) * 4
         q[:, i::8] = (((words >> shift) & 0xF).astype(np.int16) - 8).astype(np.int8)
     return q
+
+
+# ---------------------------------------------------------------------------- group-wise variant
+
+class GroupedWeight:
+    """A group-wise int8 weight (see ``int8mm_grouped_weight``)."""
+
+    def __init__(self, buf: torch.Tensor, st: _abi.GroupedWeight):
+        self.buf = buf
+        self.struct = st
+        self.K, self.N, self.G, self.n_keep = st.K, st.N, st.G, st.n_keep
+
+    @property
+    def wq(self) -> torch.Tensor:           # N x K int8
+        return _view(self.buf, self.struct.wq, self.N * self.K, torch.int8, (self.N, self.K))
+
+    @property
+    def col_absmax(self) -> torch.Tensor:   # (K/G) x N float32
+        ng = self.K // self.G
+        return _view(self.buf, self.struct.col_absmax, ng * self.N, torch.float32, (ng, self.N))
+
+    @property
+    def w_keep(self) -> torch.Tensor:
+        return _view(self.buf, self.struct.w_keep, self.n_keep * self.N, torch.float16, (self.n_keep, self.N))
+
+    @property
+    def keep_idx(self) -> torch.Tensor:
+        return _view(self.buf, self.struct.keep_idx, self.n_keep, torch.int32)
+
+
+def prepare_weight_grouped(W: torch.Tensor, G: int, keep_idx=(), stream=None) -> GroupedWeight:
+    """Convert a K x N fp16 CUDA weight to int8 with one constant per output
+    column and group of G consecutive k (once, at load)."""
+    lib = _abi.load()
+    if not (W.is_cuda and W.dtype == torch.float16 and W.dim() == 2 and W.is_contiguous()):
+        raise ValueError("W must be a contiguous 2-D float16 CUDA tensor (K x N)")
+    K, N = W.shape
+    keep = np.unique(np.asarray(keep_idx, dtype=np.int64).ravel()).astype(np.int32)
+    nbytes = lib.int8mm_grouped_weight_bytes(K, N, int(G), int(keep.size))
+    if nbytes == 0:
+        raise Int8mmError(1, f"int8mm_grouped_weight_bytes(K={K}, N={N}, G={G}, n_keep={keep.size})")
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    st = _abi.GroupedWeight()
+    kp = keep.ctypes.data_as(ctypes.c_void_p) if keep.size else None
+    with torch.cuda.device(W.device):
+        _abi.check(lib.int8mm_prepare_weight_grouped(ctypes.c_void_p(W.data_ptr()), K, N, int(G), kp, int(keep.size),
+                                                     ctypes.c_void_p(buf.data_ptr()), nbytes, ctypes.byref(st),
+                                                     _stream(stream)), "int8mm_prepare_weight_grouped")
+    return GroupedWeight(buf, st)
+
+
+def forward_grouped(X: torch.Tensor, w: GroupedWeight, threshold: float = 6.0, *, max_outliers: int | None = None,
+                    out: torch.Tensor | None = None, workspace: Workspace | None = None,
+                    acc_out: torch.Tensor | None = None, wait_limit_ns: int = 0, test_flags: int = 0,
+                    stream=None) -> torch.Tensor:
+    """Y = X W by the group-wise method (X: M x K fp16 on the weight's device).
+    acc_out (M x N x K/G int32), if given, receives the per-group int32 sums."""
+    lib = _abi.load()
+    if X.dtype != torch.float16 or X.dim() != 2 or X.shape[1] != w.K or not X.is_cuda or not X.is_contiguous():
+        raise ValueError(f"X must be a contiguous float16 CUDA tensor of shape (M, {w.K})")
+    M = X.shape[0]
+    if workspace is None:
+        workspace = Workspace(M, w.K, w.N, max_outliers, device=X.device, G=w.G)
+    if (workspace.M, workspace.K, workspace.N, workspace.G) != (M, w.K, w.N, w.G):
+        raise ValueError("workspace was made for another shape or group size")
+    Y = out if out is not None else torch.empty(M, w.N, dtype=torch.float16, device=X.device)
+    opts = _abi.ForwardOpts(0, ctypes.c_void_p(acc_out.data_ptr()) if acc_out is not None else None,
+                            int(wait_limit_ns), None, None, int(test_flags))
+    with torch.cuda.device(X.device):
+        _abi.check(lib.int8mm_forward_grouped(ctypes.c_void_p(X.data_ptr()), M, ctypes.byref(w.struct),
+                                              float(threshold), workspace.max_outliers, ctypes.c_void_p(Y.data_ptr()),
+                                              ctypes.c_void_p(workspace.buf.data_ptr()), workspace.nbytes,
+                                              ctypes.byref(opts), _stream(stream)), "int8mm_forward_grouped")
+    return Y

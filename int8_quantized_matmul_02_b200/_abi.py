@@ -32,6 +32,8 @@ EXPORTS = (
     "int8mm_forward_decode_noalloc", "int8mm_noalloc_device_status",
     "int8mm_block_quantize", "int8mm_block_dequantize",
     "int8mm_int4_weight_bytes", "int8mm_prepare_weight_int4", "int8mm_forward_int4",
+    "int8mm_grouped_weight_bytes", "int8mm_prepare_weight_grouped", "int8mm_grouped_workspace_bytes",
+    "int8mm_grouped_workspace_view_get", "int8mm_forward_grouped",
 )
 
 
@@ -44,6 +46,14 @@ class Int8mmError(RuntimeError):
 class Weight(ctypes.Structure):
     _fields_ = [
         ("K", ctypes.c_int32), ("N", ctypes.c_int32), ("n_keep", ctypes.c_int32),
+        ("wq", ctypes.c_void_p), ("col_absmax", ctypes.c_void_p), ("w_keep", ctypes.c_void_p),
+        ("keep_idx", ctypes.c_void_p), ("keep_slot", ctypes.c_void_p),
+    ]
+
+
+class GroupedWeight(ctypes.Structure):
+    _fields_ = [
+        ("K", ctypes.c_int32), ("N", ctypes.c_int32), ("G", ctypes.c_int32), ("n_keep", ctypes.c_int32),
         ("wq", ctypes.c_void_p), ("col_absmax", ctypes.c_void_p), ("w_keep", ctypes.c_void_p),
         ("keep_idx", ctypes.c_void_p), ("keep_slot", ctypes.c_void_p),
     ]
@@ -119,6 +129,17 @@ def load(path: str | None = None):
     lib.int8mm_prepare_weight_int4.restype = I
     lib.int8mm_forward_int4.argtypes = [P, I, ctypes.POINTER(Int4Weight), P, P, P]
     lib.int8mm_forward_int4.restype = I
+    lib.int8mm_grouped_weight_bytes.argtypes = [I, I, I, I]
+    lib.int8mm_grouped_weight_bytes.restype = S
+    lib.int8mm_prepare_weight_grouped.argtypes = [P, I, I, I, P, I, P, S, ctypes.POINTER(GroupedWeight), P]
+    lib.int8mm_prepare_weight_grouped.restype = I
+    lib.int8mm_grouped_workspace_bytes.argtypes = [I, I, I, I, I]
+    lib.int8mm_grouped_workspace_bytes.restype = S
+    lib.int8mm_grouped_workspace_view_get.argtypes = [P, S, I, I, I, I, I, ctypes.POINTER(WorkspaceView)]
+    lib.int8mm_grouped_workspace_view_get.restype = I
+    lib.int8mm_forward_grouped.argtypes = [P, I, ctypes.POINTER(GroupedWeight), F, I, P, P, S,
+                                           ctypes.POINTER(ForwardOpts), P]
+    lib.int8mm_forward_grouped.restype = I
     if path is None:
         _lib = lib
     return lib

@@ -71,7 +71,7 @@ struct DecodeParams {
     int num_clusters;           // cluster c owns tiles [c * num_tiles / num_clusters, (c + 1) * ...)
     int cluster, stages, groups;  // groups = ceil(M / 8)
     uint32_t tmem_cols;         // 32 columns per tile of the largest tile range, a power of two >= 32
-    uint32_t off_xq, off_mask, off_pre, off_xo, off_oslot, off_red, off_bars;  // shared-memory offsets
+    uint32_t off_xq, off_mask, off_pre, off_list, off_xo, off_oslot, off_red, off_bars;  // shared-memory offsets
 };
 
 constexpr int kDecSmemOutliers = 64;         // outlier columns whose x values are staged in shared memory
@@ -126,6 +126,16 @@ __device__ __forceinline__ uint2 dec_quant8(uint4 v, uint32_t fl, float scale) {
         hi &= mhi;
     }
     return make_uint2(lo, hi);
+}
+
+// 16-byte read-only load as a volatile instruction: issued once and kept in
+// registers (the compiler may neither repeat nor sink it).
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
 }
 
 // Pass (a) works on packed fp16 pairs with the native half2 compare and max:
@@ -187,6 +197,7 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
     uint8_t* sxq = smem + p.off_xq;
     uint32_t* smask = reinterpret_cast<uint32_t*>(smem + p.off_mask);
     int* spre = reinterpret_cast<int*>(smem + p.off_pre);
+    uint16_t* slist = reinterpret_cast<uint16_t*>(smem + p.off_list);  // [kDecSmemOutliers] outlier columns
     uint16_t* sxo = reinterpret_cast<uint16_t*>(smem + p.off_xo);  // [kDecSmemOutliers][16] fp16 x values
     int* soslot = reinterpret_cast<int*>(smem + p.off_oslot);      // [kDecSmemOutliers] kept-row slot
     uint32_t* sred = reinterpret_cast<uint32_t*>(smem + p.off_red);  // [CL-1][128][RS] peers' partial sums of the owned tile
@@ -203,6 +214,8 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
     unsigned* sra_bits = reinterpret_cast<unsigned*>(tmem_slot + 2);  // [16] row absmax (fp16 bits)
     int* sflag = reinterpret_cast<int*>(tmem_slot + 18);              // [1] total outliers
     float* srs = reinterpret_cast<float*>(tmem_slot + 20);            // [16] ra / 127^2
+    uint32_t* sown = tmem_slot + 36;                                  // [16] this CTA's row maxima
+    uint32_t* swmax = tmem_slot + 52;                                 // [10][16] per-warp row maxima
     const uint16_t* __restrict__ Xg = p.X;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -369,7 +382,7 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
 #pragma unroll
         for (int i = 0; i < kP; ++i) {
             const int c = c0 + (pt + i * kPro) / kR;
-            if (i < nit && row_ok && c < c1) xv[i] = __ldg(reinterpret_cast<const uint4*>(Xg + (size_t)prow * K) + c);
+            if (i < nit && row_ok && c < c1) xv[i] = ld_nc_v4(reinterpret_cast<const uint4*>(Xg + (size_t)prow * K) + c);
         }
         {
             // in phases over the iterations, so that their dependency chains
@@ -387,26 +400,46 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
                 for (int i = 0; i < kP; ++i)
                     if (i < nit) cfl[i] |= __shfl_xor_sync(0xffffffffu, cfl[i], off);
             }
+            // A warp's lanes hold 32 / kR consecutive chunks of one iteration,
+            // starting at a multiple of 32 / kR (c0, kPro and the warp's first
+            // pair are multiples of 32): with kR = 8 that is one whole flag word,
+            // which lane 0 stores; with kR = 16, half a word (two warps OR it).
 #pragma unroll
             for (int i = 0; i < kP; ++i) {
+                if (i >= nit) continue;
                 const int c = c0 + (pt + i * kPro) / kR;
-                if (i < nit && c < c1) {
-                    if (prow == 0 && cfl[i]) atomicOr(&smask[c >> 2], cfl[i] << ((c & 3) * 8));
-                    if (row_ok) rmax2 = __hmax2(rmax2, inlier_max8(abs8(xv[i]), cfl[i]));
+                uint32_t word = (c < c1 ? cfl[i] : 0u) << ((lane / kR) * 8);
+#pragma unroll
+                for (int off = kR; off < 32; off <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, off);
+                const int cw = c - lane / kR;  // the warp's first chunk
+                if (lane == 0 && cw < c1) {
+                    if (kR == 8) smask[cw >> 2] = word << ((cw & 3) * 8);
+                    else if (word) atomicOr(&smask[cw >> 2], word << ((cw & 3) * 8));
                 }
+                if (row_ok && c < c1) rmax2 = __hmax2(rmax2, inlier_max8(abs8(xv[i]), cfl[i]));
             }
             // non-negative fp16 bit patterns order like their values
             const uint32_t rb = as_u32(rmax2);
             uint32_t rmax = max(rb & 0xFFFFu, rb >> 16);
 #pragma unroll
             for (int off = kR; off < 32; off <<= 1) rmax = max(rmax, __shfl_xor_sync(0xffffffffu, rmax, off));
-            if (lane < kR && row_ok && rmax) atomicMax(&sra_bits[prow], rmax);
+            if (lane < kR) swmax[(warp - 2) * 16 + lane] = row_ok ? rmax : 0u;
         }
         // every X-side thread's flags and maxima are in; the mbarriers are
         // initialised and TMEM is allocated
         named_bar_sync(2, kThr);
         tc_fence_after();
         tmem_base = *tmem_slot;
+        // this CTA's row maxima from the warps' partial maxima; atomically,
+        // because a peer's maximum may already have landed in sra_bits
+        if (pt >= kPro - 16 && pt - (kPro - 16) < M) {
+            const int m = pt - (kPro - 16);
+            uint32_t v = 0u;
+#pragma unroll
+            for (int w = 0; w < kPro / 32; ++w) v = max(v, swmax[w * 16 + (m % kR)]);
+            if (v) atomicMax(&sra_bits[m], v);
+            sown[m] = v;
+        }
         // this CTA's flag words (its K range covers whole words) and row
         // maxima to every peer; the peers' arrive the same way
         if (CL > 1) {
@@ -418,7 +451,7 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
             }
             if (pt >= kPro - 16 && pt - (kPro - 16) < M) {
                 const int m = pt - (kPro - 16);
-                const uint32_t val = sra_bits[m];
+                const uint32_t val = sown[m];  // this CTA's own maximum
                 for (int q = 0; q < CL; ++q)
                     if (q != rank)
                         red_async_max_u32(map_to_rank(&sra_bits[m], (uint32_t)q), val, map_to_rank(xchg, (uint32_t)q));
@@ -482,6 +515,7 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
                 const int k = w * 32 + b;
                 if (blockIdx.x == 0) p.idx_out[s] = k;
                 if (s < kDecSmemOutliers) {
+                    slist[s] = (uint16_t)k;
                     soslot[s] = p.keep_slot[k];
 #pragma unroll
                     for (int m = 0; m < 16; ++m) sxo[s * 16 + m] = m < M ? Xg[(size_t)m * K + k] : (uint16_t)0;
@@ -510,31 +544,56 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
             for (int m = 0; m < 16; ++m) o[m] = 0.0f;
             const float cav = (owner && n < N) ? p.ca[n] : 0.0f;
             if (owner && n < N && n_eff > 0) {
-                int j = 0;
-                for (int w = 0; w < nw && j < n_eff; ++w) {
-                    uint32_t word = smask[w];
-                    while (word && j < n_eff) {
-                        const int k = w * 32 + __ffs(word) - 1;
-                        word &= word - 1;
-                        const bool staged = j < kDecSmemOutliers;
-                        const int slot = staged ? soslot[j] : p.keep_slot[k];
-                        float wv;
-                        if (slot >= 0) {
-                            wv = dec_half_to_float(p.w_keep[(size_t)slot * N + n]);
-                        } else {
-                            const float tq = __fmul_rn((float)p.wq[(size_t)n * K + k], cav);
-                            wv = __half2float(__float2half_rn(__fdiv_rn(tq, 127.0f)));
+                // the staged outliers, eight at a time: their eight weight
+                // loads are independent and in flight together
+                const int n_fast = min(n_eff, kDecSmemOutliers);
+                for (int j0 = 0; j0 < n_fast; j0 += 8) {
+                    float wv[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int j = j0 + u;
+                        wv[u] = 0.0f;
+                        if (j < n_fast) {
+                            const int slot = soslot[j];
+                            if (slot >= 0) {
+                                wv[u] = dec_half_to_float(p.w_keep[(size_t)slot * N + n]);
+                            } else {
+                                const float tq = __fmul_rn((float)p.wq[(size_t)n * K + slist[j]], cav);
+                                wv[u] = __half2float(__float2half_rn(__fdiv_rn(tq, 127.0f)));
+                            }
                         }
-                        if (staged) {
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        if (j0 + u < n_fast) {
 #pragma unroll
                             for (int m = 0; m < 16; ++m)
-                                if (m < M) o[m] = fmaf(dec_half_to_float(sxo[j * 16 + m]), wv, o[m]);
-                        } else {
+                                if (m < M) o[m] = fmaf(dec_half_to_float(sxo[(j0 + u) * 16 + m]), wv[u], o[m]);
+                        }
+                    }
+                }
+                // the rest (more outlier columns than are staged): in order,
+                // from the flag words
+                if (n_eff > n_fast) {
+                    int j = 0;
+                    for (int w = 0; w < nw && j < n_eff; ++w) {
+                        uint32_t word = smask[w];
+                        while (word && j < n_eff) {
+                            const int k = w * 32 + __ffs(word) - 1;
+                            word &= word - 1;
+                            if (j++ < n_fast) continue;
+                            const int slot = p.keep_slot[k];
+                            float wv;
+                            if (slot >= 0) {
+                                wv = dec_half_to_float(p.w_keep[(size_t)slot * N + n]);
+                            } else {
+                                const float tq = __fmul_rn((float)p.wq[(size_t)n * K + k], cav);
+                                wv = __half2float(__float2half_rn(__fdiv_rn(tq, 127.0f)));
+                            }
 #pragma unroll
                             for (int m = 0; m < 16; ++m)
                                 if (m < M) o[m] = fmaf(dec_half_to_float(Xg[(size_t)m * K + k]), wv, o[m]);
                         }
-                        ++j;
                     }
                 }
             }

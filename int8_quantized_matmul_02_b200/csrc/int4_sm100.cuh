@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(kI4Threads, 2)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = smem;
     uint8_t* sx = smem + p.off_x;
-    float* sred = reinterpret_cast<float*>(smem + p.off_red);  // [CL-1][128][RS] peers' partial sums
+    float* sred = reinterpret_cast<float*>(smem + p.off_red);  // [CL][128][RS] peers' partial sums, then its own
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bars);
     uint64_t* full = bars;
     uint64_t* empty = bars + p.stages;
@@ -330,50 +330,71 @@ __global__ void __launch_bounds__(kI4Threads, 2)
         float y[16];
 #pragma unroll
         for (int m = 0; m < 16; ++m) y[m] = 0.0f;
-        float own[16];
+        float* own = sred + (size_t)((CL - 1) * kI4TileN + ch) * RS;  // this CTA's sums of its own tile
+        // group constant (absmax) of block i for this thread's column; a half
+        // box past K (K % 256 == 128) multiplies X's zero fill, so any finite
+        // constant will do there
+        auto absmax_of = [&](int i) -> float {
+            if (i >= nb) return 0.0f;
+            const int n = (tile0 + i / nblk) * kI4TileN + ch;
+            const int g = min((kb_lo * kI4BoxK + (i % nblk) * 128) / G, ng - 1);
+            return n < N ? __ldg(p.absmax + (size_t)n * ng + g) : 0.0f;
+        };
+        // constants of the next 4 blocks load while the current 4 are drained
+        constexpr int kAhead = 4;
+        float a_next[kAhead];
 #pragma unroll
-        for (int m = 0; m < 16; ++m) own[m] = 0.0f;
+        for (int u = 0; u < kAhead; ++u) a_next[u] = absmax_of(u);
         bool ok = nb > 0;
-        for (int i = 0; ok && i < nb; ++i) {
-            const int j = i / nblk, b = i % nblk, d = i % kI4DSlots;
-            const int n = (tile0 + j) * kI4TileN + ch;
-            // a half box past K (K % 256 == 128) multiplies X's zero fill: any finite constant will do
-            const int g = min((kb_lo * kI4BoxK + b * 128) / G, ng - 1);
-            const float a = n < N ? __ldg(p.absmax + (size_t)n * ng + g) : 0.0f;
-            ok = __all_sync(0xffffffffu, wait_bounded_sleep(&dfull[d], (uint32_t)((i / kI4DSlots) & 1), wctx));
-            if (!ok) break;
-            tc_fence_after();
-            uint32_t r[16];
-            tmem_ld16(tmem_base + lane_addr + kI4DColBase + 16u * (uint32_t)d, r);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&dfree[d]);
-            const float sc = __fdiv_rn(a, 7.0f);
+        for (int i0 = 0; ok && i0 < nb; i0 += kAhead) {
+            float a_cur[kAhead];
 #pragma unroll
-            for (int m = 0; m < 16; ++m) y[m] = fmaf(__uint_as_float(r[m]), sc, y[m]);
-            if (b == nblk - 1) {
-                // tile j is complete in this K range: keep it (owner) or send it to its owner
-                if (j == rank) {
+            for (int u = 0; u < kAhead; ++u) a_cur[u] = a_next[u];
+            if (i0 + kAhead < nb) {
 #pragma unroll
-                    for (int m = 0; m < 16; ++m) own[m] = y[m];
-                } else {
-                    const int slot = rank < j ? rank : rank - 1;
-                    const uint32_t dst = map_to_rank(&sred[(size_t)(slot * kI4TileN + ch) * RS], (uint32_t)j);
-                    const uint32_t mb = map_to_rank(red_done, (uint32_t)j);
-                    st_async_v4(dst, __float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
-                                __float_as_uint(y[3]), mb);
-                    st_async_v4(dst + 16, __float_as_uint(y[4]), __float_as_uint(y[5]), __float_as_uint(y[6]),
-                                __float_as_uint(y[7]), mb);
-                    if (RS == 16) {
-                        st_async_v4(dst + 32, __float_as_uint(y[8]), __float_as_uint(y[9]), __float_as_uint(y[10]),
-                                    __float_as_uint(y[11]), mb);
-                        st_async_v4(dst + 48, __float_as_uint(y[12]), __float_as_uint(y[13]),
-                                    __float_as_uint(y[14]), __float_as_uint(y[15]), mb);
+                for (int u = 0; u < kAhead; ++u) a_next[u] = absmax_of(i0 + kAhead + u);
+            }
+#pragma unroll
+            for (int u = 0; u < kAhead; ++u) {
+                const int i = i0 + u;
+                if (i >= nb) break;
+                const int j = i / nblk, b = i % nblk, d = i % kI4DSlots;
+                ok = __all_sync(0xffffffffu, wait_bounded_sleep(&dfull[d], (uint32_t)((i / kI4DSlots) & 1), wctx));
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t r[16];
+                tmem_ld16(tmem_base + lane_addr + kI4DColBase + 16u * (uint32_t)d, r);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&dfree[d]);
+                const float sc = __fdiv_rn(a_cur[u], 7.0f);
+#pragma unroll
+                for (int m = 0; m < 16; ++m) y[m] = fmaf(__uint_as_float(r[m]), sc, y[m]);
+                if (b == nblk - 1) {
+                    // tile j is complete in this K range: keep it (owner) or send it to its owner
+                    if (j == rank) {
+#pragma unroll
+                        for (int m = 0; m < 16; ++m)
+                            if (m < RS) own[m] = y[m];
+                    } else {
+                        const int slot = rank < j ? rank : rank - 1;
+                        const uint32_t dst = map_to_rank(&sred[(size_t)(slot * kI4TileN + ch) * RS], (uint32_t)j);
+                        const uint32_t mb = map_to_rank(red_done, (uint32_t)j);
+                        st_async_v4(dst, __float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
+                                    __float_as_uint(y[3]), mb);
+                        st_async_v4(dst + 16, __float_as_uint(y[4]), __float_as_uint(y[5]), __float_as_uint(y[6]),
+                                    __float_as_uint(y[7]), mb);
+                        if (RS == 16) {
+                            st_async_v4(dst + 32, __float_as_uint(y[8]), __float_as_uint(y[9]),
+                                        __float_as_uint(y[10]), __float_as_uint(y[11]), mb);
+                            st_async_v4(dst + 48, __float_as_uint(y[12]), __float_as_uint(y[13]),
+                                        __float_as_uint(y[14]), __float_as_uint(y[15]), mb);
+                        }
                     }
-                }
 #pragma unroll
-                for (int m = 0; m < 16; ++m) y[m] = 0.0f;
+                    for (int m = 0; m < 16; ++m) y[m] = 0.0f;
+                }
             }
         }
         const int n = (tile0 + rank) * kI4TileN + ch;

@@ -16,6 +16,7 @@
 #include "codec_kernels.cuh"
 #include "decode_sm100.cuh"
 #include "gemm2sm_sm100.cuh"
+#include "gemm_grouped_sm100.cuh"
 #include "gemm_sm100.cuh"
 #include "int4_sm100.cuh"
 #include "quant_kernels.cuh"
@@ -43,6 +44,7 @@ struct DeviceInfo {
     int sm_count = 0;
     bool ok = false;
     bool attrs_set = false;
+    int cluster_cap[9] = {};  // clusters of n CTAs that fit at once with one CTA per SM (0: not asked yet)
 };
 std::mutex g_dev_mu;
 DeviceInfo g_dev[64];
@@ -81,6 +83,10 @@ int8mm_status current_device(int* dev_out, DeviceInfo** info_out) {
                                  kMaxSmemOptin) != cudaSuccess ||
             cudaFuncSetAttribute(k_decode_int8_sm100<16, 16, 384>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kMaxSmemOptin) != cudaSuccess ||
+            cudaFuncSetAttribute(k_gemm_int8_grouped<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGGSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(k_gemm_int8_grouped<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGGSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(k_int4_decode_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kMaxSmemOptin) != cudaSuccess ||
             cudaFuncSetAttribute(k_gemm_int8_2sm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -95,6 +101,37 @@ int8mm_status current_device(int* dev_out, DeviceInfo** info_out) {
     *dev_out = dev;
     *info_out = &d;
     return INT8MM_OK;
+}
+
+// Clusters of `cl` CTAs (1..8) that the device runs at once when every CTA
+// takes a whole SM: fewer than sm_count / cl when the GPCs' SM counts are not
+// multiples of cl.  Asked once per device and size, with the largest
+// shared-memory request (so one CTA per SM); sm_count / cl if the query fails.
+std::mutex g_cap_mu;
+
+int cluster_capacity(DeviceInfo* d, int cl) {
+    if (cl <= 1) return d->sm_count;
+    std::lock_guard<std::mutex> lk(g_cap_mu);
+    if (d->cluster_cap[cl] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(cl * 64));
+        cfg.blockDim = dim3(384);
+        cfg.dynamicSmemBytes = kMaxSmemOptin - 2048;
+        cudaLaunchAttribute a[1];
+        a[0].id = cudaLaunchAttributeClusterDimension;
+        a[0].val.clusterDim.x = (unsigned)cl;
+        a[0].val.clusterDim.y = 1;
+        a[0].val.clusterDim.z = 1;
+        cfg.attrs = a;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, k_decode_int8_sm100<8, 8, 384>, &cfg) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = std::max(1, d->sm_count / cl);
+        }
+        d->cluster_cap[cl] = n;
+    }
+    return d->cluster_cap[cl];
 }
 
 // ------------------------------------------------------------------ TMA descriptors
@@ -152,12 +189,33 @@ WeightLayout weight_layout(int K, int N, int n_keep) {
     return L;
 }
 
+bool grouped_ok(int K, int G) { return G >= 128 && G % 128 == 0 && K % G == 0; }
+
+// The group-wise weight: the vector-wise layout with (K/G) x N constants.
+WeightLayout grouped_weight_layout(int K, int N, int G, int n_keep) {
+    WeightLayout L{};
+    size_t o = 0;
+    L.wq = o;
+    o = align_up(o + (size_t)N * K, 256);
+    L.ca = o;
+    o = align_up(o + (size_t)N * (K / G) * 4, 256);
+    L.w_keep = o;
+    o = align_up(o + (size_t)n_keep * N * 2, 256);
+    L.keep_idx = o;
+    o = align_up(o + (size_t)n_keep * 4, 256);
+    L.keep_slot = o;
+    o = align_up(o + (size_t)K * 4, 256);
+    L.total = o;
+    return L;
+}
+
 struct WsLayout {
     size_t status, n_out, mask, idx, ra, xq, xo, wo, total;
     int kp;
 };
 
-WsLayout ws_layout(int M, int K, int N, int max_outliers) {
+// ng: constants per row of X (1 vector-wise, K / G group-wise)
+WsLayout ws_layout(int M, int K, int N, int max_outliers, int ng = 1) {
     WsLayout L{};
     L.kp = (max_outliers + 63) / 64 * 64;
     size_t o = 0;
@@ -169,7 +227,7 @@ WsLayout ws_layout(int M, int K, int N, int max_outliers) {
     L.idx = o;
     o = align_up(o + (size_t)K * 4, 256);
     L.ra = o;
-    o = align_up(o + (size_t)M * 4, 256);
+    o = align_up(o + (size_t)M * ng * 4, 256);
     L.xq = o;
     o = align_up(o + (size_t)M * K, 256);
     L.xo = o;
@@ -256,14 +314,17 @@ uint32_t fp16_threshold_bits2(float thr) {
 struct DecodePlan {
     int threads, cluster, clusters, max_tiles, stages, groups, grid, mr;  // mr: rows per chunk group (8 or 16)
     uint32_t tmem_cols;
-    uint32_t off_xq, off_mask, off_pre, off_xo, off_oslot, off_red, off_bars, bytes;
+    uint32_t off_xq, off_mask, off_pre, off_list, off_xo, off_oslot, off_red, off_bars, bytes;
 };
 
 // (chunk, row) pairs each X-side thread holds in registers (template kP of
 // the kernel): rows per chunk group 8 -> 8 pairs, 16 -> 16 pairs.
 constexpr int decode_pairs(int mr) { return mr == 8 ? 8 : 16; }
 
-bool decode_plan_shape(int M, int K, int N, int sms, int threads, size_t smem_cap, int min_stages, DecodePlan* P) {
+// dev == nullptr: no device limit on the number of clusters (only asks
+// whether the shape fits the kernel at all).
+bool decode_plan_shape(int M, int K, int N, DeviceInfo* dev, int threads, size_t smem_cap, int min_stages,
+                       DecodePlan* P) {
     const int kbt = cdiv(K, 128);
     const int mr = M <= 8 ? 8 : 16;
     const int chunks_max = decode_pairs(mr) * (threads - 64) / mr;  // 8-column chunks of X one CTA holds
@@ -273,9 +334,11 @@ bool decode_plan_shape(int M, int K, int N, int sms, int threads, size_t smem_ca
     for (int c : {4, 8}) {
         const int cl = std::min(c, kbt);
         if (cdiv(kbt, cl) * 16 > chunks_max) continue;
-        // clusters: one CTA per SM when the tiles allow (at most cl tiles per
-        // cluster), else as many waves as needed with cl tiles per cluster
-        int ncl = std::max(1, std::min(tiles, sms / cl));
+        // clusters: one CTA per SM in one wave when the tiles allow (at most
+        // cl tiles per cluster), else as many waves as needed with cl tiles
+        // per cluster
+        const int cap = dev ? cluster_capacity(dev, cl) : (1 << 20);
+        int ncl = std::max(1, std::min(tiles, cap));
         if (cdiv(tiles, ncl) > cl) ncl = cdiv(tiles, cl);
         const int tmax = cdiv(tiles, ncl);
         uint32_t tcols = 32;
@@ -283,12 +346,14 @@ bool decode_plan_shape(int M, int K, int N, int sms, int threads, size_t smem_ca
         const size_t xq = (size_t)(cdiv(kbt, cl) * groups + 1) * 1024;
         const size_t mask = align_up((size_t)nw * 4, 16);
         const size_t pre = align_up((size_t)nw * 4, 16);
+        const size_t list = (size_t)kDecSmemOutliers * 2;
         const size_t xo = (size_t)kDecSmemOutliers * 16 * 2;
         const size_t oslot = (size_t)kDecSmemOutliers * 4;
         const size_t red = (size_t)(cl - 1) * kDecTileN * 8 * groups * 4;  // one partial-sum slot per peer
-        const size_t fixed = xq + mask + pre + xo + oslot + red;
+        const size_t fixed = xq + mask + pre + list + xo + oslot + red;
         for (int s = 16; s >= min_stages; --s) {
-            const size_t bars = (size_t)(2 * s + kDecMaxTiles + 4) * 8 + 256;  // + TMEM address, abort flag, row maxima, count, scales
+            // + TMEM address, abort flag, row maxima, count, scales, own and per-warp row maxima
+            const size_t bars = (size_t)(2 * s + kDecMaxTiles + 4) * 8 + 1024;
             const size_t total = 1024 + (size_t)s * kDecStageBytes + fixed + bars;
             if (total > smem_cap) continue;
             P->threads = threads;
@@ -307,6 +372,8 @@ bool decode_plan_shape(int M, int K, int N, int sms, int threads, size_t smem_ca
             o += mask;
             P->off_pre = (uint32_t)o;
             o += pre;
+            P->off_list = (uint32_t)o;
+            o += list;
             P->off_xo = (uint32_t)o;
             o += xo;
             P->off_oslot = (uint32_t)o;
@@ -323,10 +390,10 @@ bool decode_plan_shape(int M, int K, int N, int sms, int threads, size_t smem_ca
 
 // False when (M, K) does not fit the kernel: M > 16, or a CTA's K range wider
 // than its X-side threads hold in registers even in clusters of 8.
-bool decode_plan(int M, int K, int N, int sms, DecodePlan* P) {
+bool decode_plan(int M, int K, int N, DeviceInfo* dev, DecodePlan* P) {
     if (M < 1 || M > kMaxDecodeRows) return false;
-    return decode_plan_shape(M, K, N, sms, 256, kDecSmallSmem, 4, P) ||
-           decode_plan_shape(M, K, N, sms, 384, kMaxSmemOptin, 4, P);
+    return decode_plan_shape(M, K, N, dev, 256, kDecSmallSmem, 4, P) ||
+           decode_plan_shape(M, K, N, dev, 384, kMaxSmemOptin, 4, P);
 }
 
 // Parameters of one decode launch (the workspace pointers are the caller's).
@@ -354,6 +421,7 @@ DecodeParams decode_params(const uint16_t* X, int M, const int8mm_weight* w, flo
     p.off_xq = dp.off_xq;
     p.off_mask = dp.off_mask;
     p.off_pre = dp.off_pre;
+    p.off_list = dp.off_list;
     p.off_xo = dp.off_xo;
     p.off_oslot = dp.off_oslot;
     p.off_red = dp.off_red;
@@ -404,7 +472,7 @@ struct Int4Plan {
     uint32_t tmem_cols, off_x, off_red, off_bars, bytes;
 };
 
-bool int4_plan(int M, int K, int N, int sms, Int4Plan* P) {
+bool int4_plan(int M, int K, int N, DeviceInfo* dev, Int4Plan* P) {
     if (M < 1 || M > kInt4MaxRows) return false;
     const int kbt = cdiv(K, kI4BoxK);
     const int tiles = cdiv(N, kI4TileN);
@@ -412,10 +480,10 @@ bool int4_plan(int M, int K, int N, int sms, Int4Plan* P) {
     for (size_t cap : {(size_t)kDecSmallSmem, (size_t)kMaxSmemOptin}) {
         for (int c : {4, 8}) {
             const int cl = std::min(c, kbt);
-            int ncl = std::max(1, std::min(tiles, sms / cl));
+            int ncl = std::max(1, std::min(tiles, cluster_capacity(dev, cl)));
             if (cdiv(tiles, ncl) > cl) ncl = cdiv(tiles, cl);
             const size_t xb = (size_t)cdiv(kbt, cl) * (kI4BoxK / 64) * xrows * 128 + 1024;  // + the row-8 overhang
-            const size_t red = (size_t)(cl - 1) * kI4TileN * xrows * 4;
+            const size_t red = (size_t)cl * kI4TileN * xrows * 4;  // a slot per peer and one for its own sums
             for (int s = 12; s >= 3; --s) {
                 const size_t bars = (size_t)(2 * s + 4 + 2 * kI4DSlots + 3) * 8 + 64;
                 const size_t total = 1024 + (size_t)s * kI4StageBytes + xb + red + bars;
@@ -554,7 +622,7 @@ int8mm_status int8mm_prepare_weight(const uint16_t* W, int K, int N, const int32
                    reinterpret_cast<unsigned*>(w.col_absmax));
     }
     if (e == cudaSuccess)
-        e = launch(k_quant_weight, dim3(cdiv(N, 64), cdiv(K, 64)), dim3(256), 0, s, false, W, K, N,
+        e = launch(k_quant_weight, dim3(cdiv(N, 64), cdiv(K, 64)), dim3(256), 0, s, false, W, K, N, K,
                    (const float*)w.col_absmax, w.wq);
     if (e == cudaSuccess && n_keep > 0)
         e = cudaMemcpyAsync(w.keep_idx, keep_idx_host, (size_t)n_keep * 4, cudaMemcpyHostToDevice, s);
@@ -633,7 +701,7 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
 
     // whether the decode kernel fits does not depend on the device; its grid does
     DecodePlan dp{};
-    const bool decode_fits = decode_plan(M, K, N, 1 << 20, &dp);
+    const bool decode_fits = decode_plan(M, K, N, nullptr, &dp);
     bool use_decode;
     if (path == INT8MM_PATH_DECODE) {
         if (!decode_fits) return INT8MM_ERR_INVALID_ARGUMENT;
@@ -647,7 +715,7 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
     DeviceInfo* info;
     int8mm_status st = current_device(&dev, &info);
     if (st != INT8MM_OK) return st;
-    if (use_decode && !decode_plan(M, K, N, info->sm_count, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (use_decode && !decode_plan(M, K, N, info, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* b = static_cast<uint8_t*>(ws);
@@ -714,7 +782,7 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
     }
     if (e == cudaSuccess)
         e = launch(k_gather_wo, dim3(cdiv(N, 64)), dim3(256), 0, s, true, (const int8_t*)w->wq,
-                   (const float*)w->col_absmax, (const uint16_t*)w->w_keep, (const int32_t*)w->keep_slot, K, N,
+                   (const float*)w->col_absmax, (const uint16_t*)w->w_keep, (const int32_t*)w->keep_slot, K, N, K,
                    (const int32_t*)idx, (const int32_t*)n_out, max_outliers, kp, wo, mask);
     if (e == cudaSuccess) {
         const bool pair = (path != INT8MM_PATH_GEMM_1SM) && M > kGemmBM;
@@ -792,13 +860,13 @@ int8mm_status int8mm_forward_decode_noalloc(const uint16_t* X, int M, const int8
     const NoAllocLayout L = noalloc_layout(M, K);
     if (L.total > kNoAllocBytes) return INT8MM_ERR_INVALID_ARGUMENT;
     DecodePlan dp{};
-    if (!decode_plan(M, K, N, 1 << 20, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!decode_plan(M, K, N, nullptr, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
 
     int dev;
     DeviceInfo* info;
     int8mm_status st = current_device(&dev, &info);
     if (st != INT8MM_OK) return st;
-    if (!decode_plan(M, K, N, info->sm_count, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!decode_plan(M, K, N, info, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
     uint8_t* b = nullptr;
     st = noalloc_scratch(dev, &b);
     if (st != INT8MM_OK) return st;
@@ -912,7 +980,7 @@ int8mm_status int8mm_forward_int4(const uint16_t* X, int M, const int8mm_int4_we
     int8mm_status st = current_device(&dev, &info);
     if (st != INT8MM_OK) return st;
     Int4Plan pl{};
-    if (!int4_plan(M, K, N, info->sm_count, &pl)) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!int4_plan(M, K, N, info, &pl)) return INT8MM_ERR_INVALID_ARGUMENT;
     CUtensorMap tm_w, tm_x;
     if (!make_map(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, (uint64_t)K / 2, N, (uint64_t)K / 2, 128, kI4TileN) ||
         !make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, K, M, (uint64_t)K * 2, 64, pl.xrows))
@@ -939,6 +1007,189 @@ int8mm_status int8mm_forward_int4(const uint16_t* X, int M, const int8mm_int4_we
     p.off_bars = pl.off_bars;
     return cuda_status(launch_ex(k_int4_decode_sm100, dim3(pl.grid), dim3(kI4Threads), pl.bytes,
                                  reinterpret_cast<cudaStream_t>(stream), true, pl.cluster, tm_w, tm_x, p));
+}
+
+size_t int8mm_grouped_weight_bytes(int K, int N, int G, int n_keep) {
+    if (!shape_ok(1, K, N) || !grouped_ok(K, G) || n_keep < 0 || n_keep > K) return 0;
+    return grouped_weight_layout(K, N, G, n_keep).total;
+}
+
+int8mm_status int8mm_prepare_weight_grouped(const uint16_t* W, int K, int N, int G, const int32_t* keep_idx_host,
+                                            int n_keep, void* buf, size_t buf_bytes, int8mm_grouped_weight* out,
+                                            void* stream) {
+    if (!W || !buf || !out || !shape_ok(1, K, N) || !grouped_ok(K, G) || n_keep < 0 || n_keep > K ||
+        (n_keep > 0 && !keep_idx_host))
+        return INT8MM_ERR_INVALID_ARGUMENT;
+    for (int i = 0; i < n_keep; ++i) {
+        const int k = keep_idx_host[i];
+        if (k < 0 || k >= K || (i > 0 && k <= keep_idx_host[i - 1])) return INT8MM_ERR_INVALID_ARGUMENT;
+    }
+    if (!aligned(W, 16) || !aligned(buf, 256)) return INT8MM_ERR_MISALIGNED;
+    const WeightLayout L = grouped_weight_layout(K, N, G, n_keep);
+    if (buf_bytes < L.total) return INT8MM_ERR_WORKSPACE_TOO_SMALL;
+    int dev;
+    DeviceInfo* info;
+    int8mm_status st = current_device(&dev, &info);
+    if (st != INT8MM_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* b = static_cast<uint8_t*>(buf);
+    int8mm_grouped_weight w{};
+    w.K = K;
+    w.N = N;
+    w.G = G;
+    w.n_keep = n_keep;
+    w.wq = reinterpret_cast<int8_t*>(b + L.wq);
+    w.col_absmax = reinterpret_cast<float*>(b + L.ca);
+    w.w_keep = reinterpret_cast<uint16_t*>(b + L.w_keep);
+    w.keep_idx = reinterpret_cast<int32_t*>(b + L.keep_idx);
+    w.keep_slot = reinterpret_cast<int32_t*>(b + L.keep_slot);
+    std::vector<int32_t> slot(K, -1);
+    for (int i = 0; i < n_keep; ++i) slot[keep_idx_host[i]] = i;
+    cudaError_t e = launch(k_col_absmax_grouped, dim3(cdiv(N, 2048), K / G), dim3(256), 0, s, false, W, K, N, G,
+                           w.col_absmax);
+    if (e == cudaSuccess)
+        e = launch(k_quant_weight, dim3(cdiv(N, 64), cdiv(K, 64)), dim3(256), 0, s, false, W, K, N, G,
+                   (const float*)w.col_absmax, w.wq);
+    if (e == cudaSuccess && n_keep > 0)
+        e = cudaMemcpyAsync(w.keep_idx, keep_idx_host, (size_t)n_keep * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(w.keep_slot, slot.data(), (size_t)K * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && n_keep > 0)
+        e = launch(k_copy_keep_rows, dim3(n_keep), dim3(256), 0, s, false, W, N, (const int32_t*)w.keep_idx,
+                   w.w_keep);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);  // the host arrays above go out of scope
+    if (e != cudaSuccess) return cuda_status(e);
+    *out = w;
+    return INT8MM_OK;
+}
+
+size_t int8mm_grouped_workspace_bytes(int M, int K, int N, int G, int max_outliers) {
+    if (!shape_ok(M, K, N) || !grouped_ok(K, G) || max_outliers < 0 || max_outliers > K) return 0;
+    return ws_layout(M, K, N, max_outliers, K / G).total;
+}
+
+int8mm_status int8mm_grouped_workspace_view_get(void* ws, size_t ws_bytes, int M, int K, int N, int G,
+                                                int max_outliers, int8mm_workspace_view* out) {
+    if (!ws || !out || !shape_ok(M, K, N) || !grouped_ok(K, G) || max_outliers < 0 || max_outliers > K)
+        return INT8MM_ERR_INVALID_ARGUMENT;
+    const WsLayout L = ws_layout(M, K, N, max_outliers, K / G);
+    if (ws_bytes < L.total) return INT8MM_ERR_WORKSPACE_TOO_SMALL;
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    out->status = reinterpret_cast<int32_t*>(b + L.status);
+    out->n_outliers = reinterpret_cast<int32_t*>(b + L.n_out);
+    out->outlier_idx = reinterpret_cast<int32_t*>(b + L.idx);
+    out->row_absmax = reinterpret_cast<float*>(b + L.ra);
+    out->xq = reinterpret_cast<int8_t*>(b + L.xq);
+    out->xo = reinterpret_cast<uint16_t*>(b + L.xo);
+    out->kp = L.kp;
+    return INT8MM_OK;
+}
+
+int8mm_status int8mm_forward_grouped(const uint16_t* X, int M, const int8mm_grouped_weight* w, float threshold,
+                                     int max_outliers, uint16_t* Y, void* ws, size_t ws_bytes,
+                                     const int8mm_forward_opts* opts, void* stream) {
+    if (!X || !w || !Y || !ws || !w->wq || !w->col_absmax || !w->keep_slot) return INT8MM_ERR_INVALID_ARGUMENT;
+    const int K = w->K, N = w->N, G = w->G;
+    if (!shape_ok(M, K, N) || !grouped_ok(K, G) || max_outliers < 0 || max_outliers > K)
+        return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!(threshold > 0.0f)) return INT8MM_ERR_INVALID_ARGUMENT;
+    int32_t* acc_out = opts ? opts->acc_out : nullptr;
+    cudaEvent_t ev0 = opts ? reinterpret_cast<cudaEvent_t>(opts->main_start_event) : nullptr;
+    cudaEvent_t ev1 = opts ? reinterpret_cast<cudaEvent_t>(opts->main_stop_event) : nullptr;
+    if ((ev0 == nullptr) != (ev1 == nullptr)) return INT8MM_ERR_INVALID_ARGUMENT;
+    const bool timed = ev0 != nullptr;
+    const uint32_t test_flags = opts ? opts->test_flags : 0u;
+    const uint64_t wait_ns = (opts && opts->wait_limit_ns) ? opts->wait_limit_ns : kDefaultWaitNs;
+    if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ws, 256) || !aligned(w->wq, 256) ||
+        (acc_out && !aligned(acc_out, 16)))
+        return INT8MM_ERR_MISALIGNED;
+    const int ng = K / G;
+    const WsLayout L = ws_layout(M, K, N, max_outliers, ng);
+    if (ws_bytes < L.total) return INT8MM_ERR_WORKSPACE_TOO_SMALL;
+    int dev;
+    DeviceInfo* info;
+    int8mm_status st = current_device(&dev, &info);
+    if (st != INT8MM_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    int* status = reinterpret_cast<int*>(b + L.status);
+    int32_t* n_out = reinterpret_cast<int32_t*>(b + L.n_out);
+    uint32_t* mask = reinterpret_cast<uint32_t*>(b + L.mask);
+    int32_t* idx = reinterpret_cast<int32_t*>(b + L.idx);
+    float* ra = reinterpret_cast<float*>(b + L.ra);
+    int8_t* xq = reinterpret_cast<int8_t*>(b + L.xq);
+    uint16_t* xo = reinterpret_cast<uint16_t*>(b + L.xo);
+    uint16_t* wo = reinterpret_cast<uint16_t*>(b + L.wo);
+    const int kp = L.kp;
+
+    CUtensorMap tm_a, tm_b, tm_xo, tm_wo, tm_y;
+    if (!make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, M, K, 128, 128) ||
+        !make_map(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq, K, N, K, 128, 64) ||
+        !make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Y, N, M, (uint64_t)N * 2, 64, 32))
+        return INT8MM_ERR_CUDA;
+    if (kp > 0) {
+        if (!make_map(&tm_xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xo, kp, M, (uint64_t)kp * 2, 64, 128) ||
+            !make_map(&tm_wo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wo, kp, N, (uint64_t)kp * 2, 64, 64))
+            return INT8MM_ERR_CUDA;
+    } else {
+        tm_xo = tm_a;  // never dereferenced: no outlier slices without capacity
+        tm_wo = tm_b;
+    }
+    const int sms = info->sm_count;
+    cudaError_t e;
+    {
+        const int gx = cdiv(K, 256);
+        int gy = std::max(1, std::min(cdiv(M, 8), cdiv(4 * sms, gx)));
+        int rows = cdiv(M, gy);
+        rows = (rows + 7) / 8 * 8;
+        gy = cdiv(M, rows);
+        e = launch(k_detect, dim3(gx, gy), dim3(256), 0, s, false, X, M, K, threshold, rows, mask);
+    }
+    if (e == cudaSuccess) {
+        const size_t smem = (size_t)cdiv(K, 32) * 2 * 4;
+        const long long items = (long long)M * ng;
+        const int grid = (int)std::max<long long>(1, std::min<long long>(cdiv(items, 8), (long long)sms * 4));
+        e = launch(k_quant_rows_grouped, dim3(grid), dim3(256), smem, s, true, X, M, K, G, (const uint32_t*)mask,
+                   max_outliers, kp, xq, ra, xo, idx, n_out, status);
+    }
+    if (e == cudaSuccess)
+        e = launch(k_gather_wo, dim3(cdiv(N, 64)), dim3(256), 0, s, true, (const int8_t*)w->wq,
+                   (const float*)w->col_absmax, (const uint16_t*)w->w_keep, (const int32_t*)w->keep_slot, K, N, G,
+                   (const int32_t*)idx, (const int32_t*)n_out, max_outliers, kp, wo, mask);
+    if (e == cudaSuccess) {
+        GroupedParams gp{};
+        GemmParams& p = gp.g;
+        p.M = M;
+        p.N = N;
+        p.K = K;
+        p.num_m_blocks = cdiv(M, kGGBM);
+        p.num_n_blocks = cdiv(N, kGGBN);
+        p.num_tiles = p.num_m_blocks * p.num_n_blocks;
+        {
+            const uint64_t band = (uint64_t)kGGBM * (uint64_t)K;
+            const int fit = (int)std::min<uint64_t>(1u << 20, (48ull << 20) / band);
+            p.group_m = std::min(std::max(8, fit), p.num_m_blocks);
+        }
+        p.kb_int8 = K / 128;
+        p.n_outliers = n_out;
+        p.cap = max_outliers;
+        p.status = status;
+        p.wait_limit_ns = wait_ns;
+        p.test_flags = test_flags;
+        gp.G = G;
+        gp.ng = ng;
+        gp.ra = ra;
+        gp.ca = w->col_absmax;
+        gp.acc_out = acc_out;
+        const int clusters = std::min(p.num_tiles, sms / 2);
+        if (timed) e = cudaEventRecord(ev0, s);
+        if (e == cudaSuccess)
+            e = acc_out ? launch_ex(k_gemm_int8_grouped<true>, dim3(2 * clusters), dim3(kGGThreads), kGGSmemBytes, s,
+                                    !timed, 2, tm_a, tm_b, tm_xo, tm_wo, tm_y, gp)
+                        : launch_ex(k_gemm_int8_grouped<false>, dim3(2 * clusters), dim3(kGGThreads), kGGSmemBytes, s,
+                                    !timed, 2, tm_a, tm_b, tm_xo, tm_wo, tm_y, gp);
+        if (e == cudaSuccess && timed) e = cudaEventRecord(ev1, s);
+    }
+    return cuda_status(e);
 }
 
 }  // extern "C"

@@ -5,6 +5,9 @@
 //   k_detect                        -- outlier feature columns of X (a)
 //   k_quant_rows                    -- row absmax int8 X without the outlier
 //                                      columns, plus the fp16 outlier columns (b)
+//   k_col_absmax_grouped /
+//   k_quant_rows_grouped            -- the same with one constant per group of G
+//                                      consecutive k (group-wise variant)
 //   k_gather_wo                     -- fp16 weight rows of the outlier dims (d)
 // All loads of X / W are 16-byte vectors along the contiguous dimension.
 #pragma once
@@ -59,9 +62,34 @@ __global__ void k_col_absmax(const uint16_t* __restrict__ W, int K, int N, int r
     }
 }
 
-// Wq[n, k] = round_half_even(W[k, n] * (127 / ca[n])), transposed through a
-// 64 x 64 shared tile.  Block 256 threads, grid (ceil(N/64), ceil(K/64)).
-__global__ void k_quant_weight(const uint16_t* __restrict__ W, int K, int N, const float* __restrict__ ca,
+// ca[g * N + n] = max over the group g of G consecutive k of |W[k, n]|.
+// Block 256 threads, each 8 consecutive columns; grid (ceil(N/2048), K/G).
+__global__ void k_col_absmax_grouped(const uint16_t* __restrict__ W, int K, int N, int G, float* __restrict__ ca) {
+    const int col0 = (blockIdx.x * 256 + threadIdx.x) * 8;
+    if (col0 >= N) return;
+    const int g = blockIdx.y;
+    uint32_t m[4] = {0, 0, 0, 0};
+    for (int k = g * G; k < (g + 1) * G; ++k) {
+        uint4 v = __ldg(reinterpret_cast<const uint4*>(W + (size_t)k * N + col0));
+        m[0] = __vmaxu2(m[0], abs_bits2(v.x));
+        m[1] = __vmaxu2(m[1], abs_bits2(v.y));
+        m[2] = __vmaxu2(m[2], abs_bits2(v.z));
+        m[3] = __vmaxu2(m[3], abs_bits2(v.w));
+    }
+    float* dst = ca + (size_t)g * N + col0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        dst[2 * i] = half_bits_to_float(m[i] & 0xFFFF);
+        dst[2 * i + 1] = half_bits_to_float(m[i] >> 16);
+    }
+}
+
+// Wq[n, k] = round_half_even(W[k, n] * (127 / ca)), transposed through a
+// 64 x 64 shared tile; ca is the constant of column n and of the group of G
+// consecutive k that holds k (ca[(k / G) * N + n]; G = K: one constant per
+// column).  G is a multiple of 64, so a tile lies in one group.  Block 256
+// threads, grid (ceil(N/64), ceil(K/64)).
+__global__ void k_quant_weight(const uint16_t* __restrict__ W, int K, int N, int G, const float* __restrict__ ca,
                                int8_t* __restrict__ Wq) {
     __shared__ uint16_t tile[64][64 + 8];
     const int n0 = blockIdx.x * 64, k0 = blockIdx.y * 64;
@@ -79,7 +107,7 @@ __global__ void k_quant_weight(const uint16_t* __restrict__ W, int K, int N, con
     const int nl = t >> 2, kl = (t & 3) * 16;
     const int n = n0 + nl;
     if (n >= N) return;
-    const float a = ca[n];
+    const float a = ca[(size_t)(k0 / G) * N + n];
     const float scale = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
     uint32_t packed[4];
 #pragma unroll
@@ -246,6 +274,59 @@ __device__ __forceinline__ uint2 quant_chunk(uint4 v, const uint32_t* smask, con
     return make_uint2(out[0], out[1]);
 }
 
+// The outlier bitmask into shared memory with the exclusive prefix counts of
+// its words (spre[w] = outlier columns before word w); returns the total.
+// Every thread of the 256-thread block calls it (it has block barriers).
+__device__ __forceinline__ int load_mask_prefix(const uint32_t* __restrict__ mask, int nw, uint32_t* smask, int* spre,
+                                                int* red) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int carry = 0;
+    for (int base = 0; base < nw; base += 256) {
+        const int w = base + tid;
+        const uint32_t word = w < nw ? mask[w] : 0u;
+        if (w < nw) smask[w] = word;
+        const int c = __popc(word);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) red[warp] = incl;
+        __syncthreads();
+        int wsum = 0, blk_total = 0;
+        for (int i = 0; i < 8; ++i) {
+            if (i < warp) wsum += red[i];
+            blk_total += red[i];
+        }
+        if (w < nw) spre[w] = carry + wsum + incl - c;
+        carry += blk_total;
+        __syncthreads();
+    }
+    return carry;
+}
+
+// Block 0's part of the row quantisers: the outlier count, the overflow flag
+// and the ascending outlier list.
+__device__ __forceinline__ void write_outlier_list(const uint32_t* smask, const int* spre, int nw, int total, int cap,
+                                                   int32_t* __restrict__ idx, int32_t* __restrict__ n_out,
+                                                   int* __restrict__ status) {
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        *n_out = total;
+        if (total > cap) atomicOr(status, kStatusOverflow);
+    }
+    for (int w = tid; w < nw; w += 256) {
+        uint32_t word = smask[w];
+        int s = spre[w];
+        while (word) {
+            const int b = __ffs(word) - 1;
+            idx[s++] = w * 32 + b;
+            word &= word - 1;
+        }
+    }
+}
+
 // Per row m: ra[m] = max over non-outlier columns of |X[m,k]|,
 // Xq[m,k] = outlier ? 0 : q(X[m,k]), Xo[m, slot(k)] = X[m,k] for outlier k,
 // with Xo zero-padded to a multiple of 64 columns.  Block 0 also writes the
@@ -270,30 +351,7 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
     pdl_wait();  // the outlier bitmask comes from k_detect
     pdl_launch_dependents();
 
-    // exclusive scan of popcounts over the mask words
-    int carry = 0;
-    for (int base = 0; base < nw; base += 256) {
-        const int w = base + tid;
-        const uint32_t word = w < nw ? mask[w] : 0u;
-        if (w < nw) smask[w] = word;
-        const int c = __popc(word);
-        int incl = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        if (lane == 31) red[warp] = incl;
-        __syncthreads();
-        int wsum = 0, blk_total = 0;
-        for (int i = 0; i < 8; ++i) {
-            if (i < warp) wsum += red[i];
-            blk_total += red[i];
-        }
-        if (w < nw) spre[w] = carry + wsum + incl - c;
-        carry += blk_total;
-        __syncthreads();
-    }
+    const int carry = load_mask_prefix(mask, nw, smask, spre, red);
     // A warp's iteration covers 256 chunks (2048 columns, 64 mask words); a
     // window with no outlier column (the common case) skips the per-chunk
     // flag lookups.
@@ -311,21 +369,7 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
     const int n_eff = min(total, cap);
     const int n_pad = min(kp, (n_eff + 63) / 64 * 64);
 
-    if (blockIdx.x == 0) {
-        if (tid == 0) {
-            *n_out = total;
-            if (total > cap) atomicOr(status, kStatusOverflow);
-        }
-        for (int w = tid; w < nw; w += 256) {
-            uint32_t word = smask[w];
-            int s = spre[w];
-            while (word) {
-                const int b = __ffs(word) - 1;
-                idx[s++] = w * 32 + b;
-                word &= word - 1;
-            }
-        }
-    }
+    if (blockIdx.x == 0) write_outlier_list(smask, spre, nw, total, cap, idx, n_out, status);
 
     for (int m = blockIdx.x * 8 + warp; m < M; m += gridDim.x * 8) {
         const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)m * K);
@@ -382,16 +426,72 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
     }
 }
 
+// Group-wise variant of k_quant_rows: one constant per row and group of G
+// consecutive columns (G a multiple of 128), ra[m * (K/G) + g] = max |X[m,k]|
+// over the non-outlier columns of the group, and the codes of the group
+// with its own scale.  One warp per (row, group) item, lanes strided over the
+// group's 8-column chunks: a first pass takes the maximum, a second (served
+// by L1/L2) writes the codes and the outlier values.  Block 0 also writes the
+// outlier list, the count and the overflow flag.  Block 256 threads.
+__global__ void __launch_bounds__(256) k_quant_rows_grouped(const uint16_t* __restrict__ X, int M, int K, int G,
+                                                            const uint32_t* __restrict__ mask, int cap, int kp,
+                                                            int8_t* __restrict__ Xq, float* __restrict__ ra,
+                                                            uint16_t* __restrict__ Xo, int32_t* __restrict__ idx,
+                                                            int32_t* __restrict__ n_out, int* __restrict__ status) {
+    extern __shared__ uint32_t qsm[];
+    const int nw = (K + 31) / 32;
+    uint32_t* smask = qsm;
+    int* spre = reinterpret_cast<int*>(qsm + nw);
+    __shared__ int red[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    pdl_wait();  // the outlier bitmask comes from k_detect
+    pdl_launch_dependents();
+    const int total = load_mask_prefix(mask, nw, smask, spre, red);
+    const int n_eff = min(total, cap);
+    const int n_pad = min(kp, (n_eff + 63) / 64 * 64);
+    if (blockIdx.x == 0) write_outlier_list(smask, spre, nw, total, cap, idx, n_out, status);
+
+    const int ng = K / G, cpg = G / 8;  // chunks per group
+    const long long items = (long long)M * ng;
+    for (long long it = (long long)blockIdx.x * 8 + warp; it < items; it += (long long)gridDim.x * 8) {
+        const int m = (int)(it / ng), g = (int)(it % ng);
+        const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)m * K);
+        const int c0 = g * cpg, c1 = c0 + cpg;
+        uint32_t amax = 0;
+        for (int c = c0 + lane; c < c1; c += 32) {
+            const uint4 v = __ldg(xr + c);
+            const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
+            amax = max(amax, fl ? chunk_inlier_absmax(v, smask, c) : chunk_absmax_h2(v));
+        }
+        amax = __reduce_max_sync(0xffffffffu, amax);
+        const float rmax = half_bits_to_float(amax);
+        const float scale = rmax > 0.0f ? __fdiv_rn(127.0f, rmax) : 0.0f;
+        if (lane == 0) ra[(size_t)m * ng + g] = rmax;
+        uint2* qr = reinterpret_cast<uint2*>(Xq + (size_t)m * K);
+        uint16_t* xo_row = Xo + (size_t)m * kp;
+        for (int c = c0 + lane; c < c1; c += 32) {
+            const uint4 v = __ldg(xr + c);
+            const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
+            qr[c] = fl ? quant_chunk(v, smask, spre, c, rmax, scale, n_eff, xo_row) : quant8_plain(v, scale);
+        }
+        if (g == 0)
+            for (int j = n_eff + lane; j < n_pad; j += 32) xo_row[j] = 0;
+    }
+}
+
 // ------------------------------------------------------------------ (d) outlier weight rows
 
 // Wo[n, j] (N x kp fp16, K-major) = the fp16 weight row of outlier j: the kept
 // row W[idx[j], n] when idx[j] was kept at preparation, else the dequantised
-// value fp16(Wq[n, idx[j]] * ca[n] / 127); zero for n_eff <= j < pad64(n_eff).
+// value fp16(Wq[n, idx[j]] * ca / 127) with the constant of column n and of
+// the group of idx[j] (ca[(k / G) * N + n]; G = K: one per column); zero for
+// n_eff <= j < pad64(n_eff).
 // Block 256 threads over 64 output channels; block 0 clears the outlier
 // bitmask for the next call.
 __global__ void __launch_bounds__(256) k_gather_wo(const int8_t* __restrict__ Wq, const float* __restrict__ ca,
                                                    const uint16_t* __restrict__ w_keep,
-                                                   const int32_t* __restrict__ keep_slot, int K, int N,
+                                                   const int32_t* __restrict__ keep_slot, int K, int N, int G,
                                                    const int32_t* __restrict__ idx,
                                                    const int32_t* __restrict__ n_out, int cap, int kp,
                                                    uint16_t* __restrict__ Wo, uint32_t* __restrict__ mask) {
@@ -424,7 +524,7 @@ __global__ void __launch_bounds__(256) k_gather_wo(const int8_t* __restrict__ Wq
                 if (slot >= 0) {
                     v = w_keep[(size_t)slot * N + n];
                 } else {
-                    float t = __fmul_rn((float)Wq[(size_t)n * K + k], ca[n]);
+                    float t = __fmul_rn((float)Wq[(size_t)n * K + k], ca[(size_t)(k / G) * N + n]);
                     v = __half_as_ushort(__float2half_rn(__fdiv_rn(t, 127.0f)));
                 }
             }

@@ -135,6 +135,10 @@ def sample_points(M: int, N: int, count: int, seed: int, tiles=((128, 256),)):
 # with 128 as the finer setting.
 INT4_GROUPS = (1024, 128)
 
+# Group-wise variant: the 175B-scale FFN shape with groups of 1024 (the group
+# size of the scite report's GPTQ snippet) and of 128 (a finer setting).
+GROUP_SIZES = (1024, 128)
+
 # Block-wise codec workload: the fp32 state of one weight of the 175B-scale FFN
 # (4096 x 12288 values), blocks of 2048.
 CODEC_N = 4096 * 12288
