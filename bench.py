@@ -1,13 +1,22 @@
 """Benchmark of the LLM.int8() matmul on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 175b]
+                    [--no-decode] [--no-variants] [--no-configs] [--no-cpu-baseline]
 
 Prints ONE JSON line.  The headline workload is the 175B-scale FFN matmul
 (X 4096 x 12288, W 12288 x 49152, 24 seeded outlier columns, threshold 6.0):
 throughput in int8 TOPS (2*M*N*K per forward, all K counted) with the
-dominant kernel's roofline against the dense-int8 tensor peak.  A "decode"
-object adds the decode-shaped FFN up-projection (X 8 x 4096, W 4096 x 11008)
-in HBM GB/s against the measured copy bandwidth.
+dominant kernel's roofline against the dense-int8 tensor peak.  Objects on the
+same line:
+  decode       the decode-shaped FFN up-projection (X 8 x 4096, W 4096 x 11008)
+               in HBM GB/s against the measured copy bandwidth, judged on
+               forwards back to back (the launch alone reported beside it);
+  configs      the prefill FFN and the attention-QKV sweep (0, 12, 48, 123
+               outlier columns and threshold = inf) in TOPS;
+  grouped      the group-wise variant at the headline shape (groups of 1024
+               and 128);
+  decode_int4  the 4-bit weight-only product on the decode workload;
+  block_codec  the block-wise 8-bit codec on a 201 MB fp32 vector.
 
 One step = one whole forward (outlier detection, X quantisation, outlier weight
 gather, int8 GEMM with fused dequantising epilogue and fp16 outlier product);

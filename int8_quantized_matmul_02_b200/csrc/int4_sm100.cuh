@@ -32,7 +32,7 @@
 // does; warp 0 streams 128 (columns) x 256 (k) boxes of packed codes through a
 // TMA ring from launch on, warps 2-5 widen each half box (128 k) to fp16 and
 // write it to tensor memory as the A operand (thread = output column =
-// TMEM lane), warp 1 issues tcgen05.mma kind::f16 with A from tensor memory
+// TMEM lane; four such operands in flight), warp 1 issues tcgen05.mma kind::f16 with A from tensor memory
 // and X (loaded once by TMA, 128-byte swizzled, K-major) as the 16-column B
 // operand into one of four fp32 accumulators, and warps 6-9 drain each
 // accumulator, scale it and add it up per column; the partial sums of a
@@ -107,8 +107,10 @@ constexpr int kI4TileN = 128;
 constexpr int kI4BoxK = 256;             // k per packed box (128 bytes per row)
 constexpr int kI4StageBytes = kI4TileN * 128;  // 16 KB
 constexpr int kI4DSlots = 4;             // fp32 accumulators in TMEM (16 columns each)
-constexpr uint32_t kI4AColBase = 0;      // two A slots of 64 columns (128 k of fp16)
-constexpr uint32_t kI4DColBase = 128;
+constexpr int kI4ASlots = 4;             // fp16 A operands in TMEM (64 columns = 128 k each)
+constexpr uint32_t kI4AColBase = 0;
+constexpr uint32_t kI4DColBase = 64 * kI4ASlots;
+constexpr uint32_t kI4TmemCols = 512;    // the whole TMEM of the SM: one CTA per SM
 
 __device__ __forceinline__ void i4_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                               uint32_t accumulate) {
@@ -134,7 +136,7 @@ __device__ __forceinline__ void i4_widen(uint32_t w, uint32_t* out) {
     }
 }
 
-__global__ void __launch_bounds__(kI4Threads, 2)
+__global__ void __launch_bounds__(kI4Threads, 1)
     k_int4_decode_sm100(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                         const Int4Params p) {
     extern __shared__ uint8_t smem_raw[];
@@ -145,9 +147,9 @@ __global__ void __launch_bounds__(kI4Threads, 2)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bars);
     uint64_t* full = bars;
     uint64_t* empty = bars + p.stages;
-    uint64_t* afull = bars + 2 * p.stages;  // [2]
-    uint64_t* afree = afull + 2;            // [2]
-    uint64_t* dfull = afree + 2;            // [4]
+    uint64_t* afull = bars + 2 * p.stages;  // [kI4ASlots]
+    uint64_t* afree = afull + kI4ASlots;    // [kI4ASlots]
+    uint64_t* dfull = afree + kI4ASlots;    // [kI4DSlots]
     uint64_t* dfree = dfull + kI4DSlots;    // [4]
     uint64_t* xfull = dfree + kI4DSlots;
     uint64_t* red_done = xfull + 1;
@@ -180,7 +182,7 @@ __global__ void __launch_bounds__(kI4Threads, 2)
                 mbar_init(&full[s], 1);
                 mbar_init(&empty[s], 4);
             }
-            for (int a = 0; a < 2; ++a) {
+            for (int a = 0; a < kI4ASlots; ++a) {
                 mbar_init(&afull[a], 4);
                 mbar_init(&afree[a], 1);
             }
@@ -248,8 +250,8 @@ __global__ void __launch_bounds__(kI4Threads, 2)
             bool ok = wait_bounded_sleep(xfull, 0, wctx), issued = false;
             tc_fence_after();
             for (int i = 0; ok && i < nb; ++i) {
-                const int a = i & 1, d = i % kI4DSlots;
-                if (!wait_bounded_sleep(&afull[a], (uint32_t)((i >> 1) & 1), wctx) ||
+                const int a = i % kI4ASlots, d = i % kI4DSlots;
+                if (!wait_bounded_sleep(&afull[a], (uint32_t)((i / kI4ASlots) & 1), wctx) ||
                     !wait_bounded_sleep(&dfree[d], (uint32_t)(((i / kI4DSlots) & 1) ^ 1), wctx)) {
                     ok = false;
                     break;
@@ -259,11 +261,11 @@ __global__ void __launch_bounds__(kI4Threads, 2)
                 const uint32_t dt = tmem_base + kI4DColBase + 16u * (uint32_t)d;
                 const uint32_t at = tmem_base + kI4AColBase + 64u * (uint32_t)a;
 #pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    // B: k = b * 128 + 16 s within the range -> X box (k / 64), 32-byte step inside it
-                    const int kk = b * 128 + 16 * s;
+                for (int st = 0; st < 8; ++st) {
+                    // B: k = b * 128 + 16 st within the range -> X box (k / 64), 32-byte step inside it
+                    const int kk = b * 128 + 16 * st;
                     const uint64_t db = db0 + (uint64_t)(((uint32_t)(kk >> 6) * xbox_bytes + (uint32_t)((kk & 63) * 2)) >> 4);
-                    i4_mma_f16_ts(dt, at + 8u * (uint32_t)s, db, idesc, s > 0 ? 1u : 0u);
+                    i4_mma_f16_ts(dt, at + 8u * (uint32_t)st, db, idesc, st > 0 ? 1u : 0u);
                 }
                 tc_commit(&afree[a]);
                 tc_commit(&dfull[d]);
@@ -281,11 +283,11 @@ __global__ void __launch_bounds__(kI4Threads, 2)
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         bool ok = true;
         for (int i = 0; ok && i < nb; ++i) {
-            const int t = i >> 1, h = i & 1, a = i & 1;
+            const int t = i >> 1, h = i & 1, a = i % kI4ASlots;
             const int stage = t % p.stages;
             const uint32_t ph = (uint32_t)((t / p.stages) & 1);
             ok = __all_sync(0xffffffffu, wait_bounded_sleep(&full[stage], ph, wctx)) &&
-                 __all_sync(0xffffffffu, wait_bounded_sleep(&afree[a], (uint32_t)(((i >> 1) & 1) ^ 1), wctx));
+                 __all_sync(0xffffffffu, wait_bounded_sleep(&afree[a], (uint32_t)(((i / kI4ASlots) & 1) ^ 1), wctx));
             if (!ok) break;
             tc_fence_after();
             const uint8_t* src = ring + stage * kI4StageBytes + row * 128;

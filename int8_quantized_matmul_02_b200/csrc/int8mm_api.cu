@@ -477,7 +477,8 @@ bool int4_plan(int M, int K, int N, DeviceInfo* dev, Int4Plan* P) {
     const int kbt = cdiv(K, kI4BoxK);
     const int tiles = cdiv(N, kI4TileN);
     const int xrows = M <= 8 ? 8 : 16;
-    for (size_t cap : {(size_t)kDecSmallSmem, (size_t)kMaxSmemOptin}) {
+    // one CTA per SM (the kernel takes the whole TMEM)
+    for (size_t cap : {(size_t)kMaxSmemOptin}) {
         for (int c : {4, 8}) {
             const int cl = std::min(c, kbt);
             int ncl = std::max(1, std::min(tiles, cluster_capacity(dev, cl)));
@@ -485,7 +486,7 @@ bool int4_plan(int M, int K, int N, DeviceInfo* dev, Int4Plan* P) {
             const size_t xb = (size_t)cdiv(kbt, cl) * (kI4BoxK / 64) * xrows * 128 + 1024;  // + the row-8 overhang
             const size_t red = (size_t)cl * kI4TileN * xrows * 4;  // a slot per peer and one for its own sums
             for (int s = 12; s >= 3; --s) {
-                const size_t bars = (size_t)(2 * s + 4 + 2 * kI4DSlots + 3) * 8 + 64;
+                const size_t bars = (size_t)(2 * s + 2 * kI4ASlots + 2 * kI4DSlots + 3) * 8 + 64;
                 const size_t total = 1024 + (size_t)s * kI4StageBytes + xb + red + bars;
                 if (total > cap) continue;
                 P->cluster = cl;
@@ -493,7 +494,7 @@ bool int4_plan(int M, int K, int N, DeviceInfo* dev, Int4Plan* P) {
                 P->stages = s;
                 P->xrows = xrows;
                 P->grid = cl * ncl;
-                P->tmem_cols = 256;
+                P->tmem_cols = kI4TmemCols;
                 size_t o = (size_t)s * kI4StageBytes;
                 P->off_x = (uint32_t)o;
                 o += xb;
@@ -774,11 +775,18 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
         e = launch(k_detect, dim3(gx, gy), dim3(256), 0, s, false, X, M, K, threshold, rows, mask);
     }
     if (e == cudaSuccess) {
-        // mask words, their prefix counts, and one flag word per 2048-column window
-        const size_t smem = ((size_t)cdiv(K, 32) * 2 + (size_t)cdiv(K, 2048)) * 4;
-        const int grid = std::max(1, std::min(cdiv(M, 8), sms * 4));
-        e = launch(k_quant_rows, dim3(grid), dim3(256), smem, s, true, X, M, K, (const uint32_t*)mask,
-                   max_outliers, kp, xq, ra, xo, idx, n_out, status);
+        if (K <= 256 * 8 * kQRChunks) {
+            // one row per block, held in registers: X read once
+            const size_t smem = (size_t)cdiv(K, 32) * 2 * 4;
+            e = launch(k_quant_rows_reg, dim3(M), dim3(256), smem, s, true, X, M, K, (const uint32_t*)mask,
+                       max_outliers, kp, xq, ra, xo, idx, n_out, status);
+        } else {
+            // mask words, their prefix counts, and one flag word per 2048-column window
+            const size_t smem = ((size_t)cdiv(K, 32) * 2 + (size_t)cdiv(K, 2048)) * 4;
+            const int grid = std::max(1, std::min(cdiv(M, 8), sms * 4));
+            e = launch(k_quant_rows, dim3(grid), dim3(256), smem, s, true, X, M, K, (const uint32_t*)mask,
+                       max_outliers, kp, xq, ra, xo, idx, n_out, status);
+        }
     }
     if (e == cudaSuccess)
         e = launch(k_gather_wo, dim3(cdiv(N, 64)), dim3(256), 0, s, true, (const int8_t*)w->wq,

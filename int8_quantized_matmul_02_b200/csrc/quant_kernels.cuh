@@ -426,6 +426,74 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
     }
 }
 
+// k_quant_rows with one row per 256-thread block, the row held in registers
+// (up to kQRChunks 8-column chunks per thread: K <= 256 * 8 * kQRChunks), so X
+// is read from memory once: the loads are issued first and land while the
+// block takes the prefix counts of the outlier bitmask; the row maximum is one
+// block reduction, and the codes go out in the same pass (each warp stores
+// 256 contiguous bytes per step).  Same results as k_quant_rows.
+constexpr int kQRChunks = 8;
+
+__global__ void __launch_bounds__(256) k_quant_rows_reg(const uint16_t* __restrict__ X, int M, int K,
+                                                        const uint32_t* __restrict__ mask, int cap, int kp,
+                                                        int8_t* __restrict__ Xq, float* __restrict__ ra,
+                                                        uint16_t* __restrict__ Xo, int32_t* __restrict__ idx,
+                                                        int32_t* __restrict__ n_out, int* __restrict__ status) {
+    extern __shared__ uint32_t qsm[];
+    const int nw = (K + 31) / 32;
+    uint32_t* smask = qsm;
+    int* spre = reinterpret_cast<int*>(qsm + nw);
+    __shared__ int red[8];
+    __shared__ uint32_t bmax[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int m = blockIdx.x;
+    const int nchunk = K / 8;
+
+    pdl_wait();  // the outlier bitmask comes from k_detect
+    pdl_launch_dependents();
+    const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)m * K);
+    uint4 v[kQRChunks];
+#pragma unroll
+    for (int i = 0; i < kQRChunks; ++i) {
+        const int c = tid + 256 * i;
+        if (c < nchunk) v[i] = __ldg(xr + c);
+    }
+    const int total = load_mask_prefix(mask, nw, smask, spre, red);
+    const int n_eff = min(total, cap);
+    const int n_pad = min(kp, (n_eff + 63) / 64 * 64);
+    if (m == 0) write_outlier_list(smask, spre, nw, total, cap, idx, n_out, status);
+
+    uint32_t amax = 0;
+#pragma unroll
+    for (int i = 0; i < kQRChunks; ++i) {
+        const int c = tid + 256 * i;
+        if (c < nchunk) {
+            const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
+            amax = max(amax, fl ? chunk_inlier_absmax(v[i], smask, c) : chunk_absmax_h2(v[i]));
+        }
+    }
+    amax = __reduce_max_sync(0xffffffffu, amax);
+    if (lane == 0) bmax[warp] = amax;
+    __syncthreads();
+    amax = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) amax = max(amax, bmax[w]);
+    const float rmax = half_bits_to_float(amax);
+    const float scale = rmax > 0.0f ? __fdiv_rn(127.0f, rmax) : 0.0f;
+    if (tid == 0) ra[m] = rmax;
+    uint2* qr = reinterpret_cast<uint2*>(Xq + (size_t)m * K);
+    uint16_t* xo_row = Xo + (size_t)m * kp;
+#pragma unroll
+    for (int i = 0; i < kQRChunks; ++i) {
+        const int c = tid + 256 * i;
+        if (c < nchunk) {
+            const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
+            qr[c] = fl ? quant_chunk(v[i], smask, spre, c, rmax, scale, n_eff, xo_row) : quant8_plain(v[i], scale);
+        }
+    }
+    for (int j = n_eff + tid; j < n_pad; j += 256) xo_row[j] = 0;
+}
+
 // Group-wise variant of k_quant_rows: one constant per row and group of G
 // consecutive columns (G a multiple of 128), ra[m * (K/G) + g] = max |X[m,k]|
 // over the non-outlier columns of the group, and the codes of the group

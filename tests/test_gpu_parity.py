@@ -97,6 +97,13 @@ def test_gemm_path_outlier_counts_production_kernel(n_seed, path):
     assert r["idx"].size >= n_seed
 
 
+@pytest.mark.parametrize("with_acc", [True, False])
+def test_gemm_path_long_rows(with_acc):
+    """K above what the row quantiser holds in registers (256 threads x 8
+    chunks of 8 columns): the two-pass row quantiser runs instead."""
+    _run_case(40, 16400, 272, 3, path="gemm", seed=61, with_acc=with_acc)
+
+
 @pytest.mark.parametrize("keep", ["none", "all"])
 def test_gemm_path_kept_and_dequantised_rows(keep):
     _run_case(130, 768, 528, 5, path="gemm", keep=keep, seed=7)
