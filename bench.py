@@ -573,6 +573,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=2000)
     ap.add_argument("--no-variants", action="store_true", help="skip the 4-bit and codec objects")
     ap.add_argument("--no-configs", action="store_true", help="skip the prefill and QKV-sweep objects")
+    ap.add_argument("--only", choices=["decode", "decode_int4", "block_codec", "grouped"],
+                    help="run one object alone (for profiling) and print it as the JSON line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -630,6 +632,24 @@ def main():
     pk, pk_kind = peaks()
 
     cap = min(args.max_outliers, wl.K)
+    if args.only:
+        # one object alone, for a profiler run: no headline, no CPU baseline
+        if args.only == "decode":
+            d = run_decode(args.decode_steps, args.warmup, dev, min(args.max_outliers, 4096))
+            out = {"us_per_step": d["plain_us"], "us_alone": d["kern_us"], "graph_us": d["graph_us"]}
+        elif args.only == "decode_int4":
+            out = {f"G{G}": run_int4_decode(args.decode_steps, args.warmup, dev, G) for G in synth.INT4_GROUPS}
+            for v in out.values():
+                v.pop("wl", None)
+        elif args.only == "block_codec":
+            out = run_codec(args.steps, args.warmup, dev)
+        else:
+            out = {}
+            for G in synth.GROUP_SIZES:
+                rg = run_grouped(wl, G, args.steps, args.warmup, dev, cap)
+                out[f"G{G}"] = {"ms_per_step": rg["total_ms"] / args.steps, "n_o": rg["n_o"]}
+        print(json.dumps({"only": args.only, "result": out}, default=str), flush=True)
+        return 0
     small = wl.M <= 16
     if small:
         r = run_decode(args.steps * 100, args.warmup, dev, cap)

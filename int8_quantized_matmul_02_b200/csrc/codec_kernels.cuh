@@ -119,4 +119,45 @@ __global__ void __launch_bounds__(256) k_block_dequant(const int8_t* __restrict_
     }
 }
 
+// Dequantisation for blocks of at least 256 values: a persistent 256-thread
+// CTA takes one block at a time, first the 129 values RN32(RN32(q * absmax) /
+// 127) for q = 0..128 into shared memory (one division each; -q gives the
+// negated value, since both roundings are symmetric), then the block's codes,
+// four per thread per step (one 32-bit load, one 16-byte store), by table
+// look-up.  Two tables alternate, so one barrier per block suffices.
+// B % 4 == 0, so a block's codes start on a 4-byte boundary.
+__global__ void __launch_bounds__(256) k_block_dequant_table(const int8_t* __restrict__ q, const float* __restrict__ absmax,
+                                                             long long n, int B, float* __restrict__ out) {
+    __shared__ float tbl[2][129];
+    const long long nblocks = (n + B - 1) / B;
+    int par = 0;
+    for (long long b = blockIdx.x; b < nblocks; b += gridDim.x) {
+        const float a = __ldg(absmax + b);
+        if (threadIdx.x < 129) tbl[par][threadIdx.x] = __fdiv_rn(__fmul_rn((float)threadIdx.x, a), 127.0f);
+        __syncthreads();  // (the other table was last read before the previous barrier)
+        const long long lo = b * (long long)B;
+        const int len = (int)min((long long)B, n - lo);
+        const float* t = tbl[par];
+        for (int e = 4 * threadIdx.x; e < len; e += 1024) {
+            if (e + 3 < len) {
+                const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(q + lo) + e / 4);
+                float4 r;
+                const int c0 = (int8_t)(w & 0xFFu), c1 = (int8_t)((w >> 8) & 0xFFu);
+                const int c2 = (int8_t)((w >> 16) & 0xFFu), c3 = (int8_t)(w >> 24);
+                r.x = c0 < 0 ? -t[-c0] : t[c0];
+                r.y = c1 < 0 ? -t[-c1] : t[c1];
+                r.z = c2 < 0 ? -t[-c2] : t[c2];
+                r.w = c3 < 0 ? -t[-c3] : t[c3];
+                *reinterpret_cast<float4*>(out + lo + e) = r;
+            } else {
+                for (int j = e; j < len; ++j) {
+                    const int c = q[lo + j];
+                    out[lo + j] = c < 0 ? -t[-c] : t[c];
+                }
+            }
+        }
+        par ^= 1;
+    }
+}
+
 }  // namespace i8mm

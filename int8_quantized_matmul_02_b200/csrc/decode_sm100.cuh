@@ -8,37 +8,27 @@
 // the first tensor-core instruction short:
 //
 // Clusters of CL CTAs (4, or 8 for long K; as many as K has 128-column blocks
-// when that is fewer) split K: CTA r of a cluster owns the r-th K range of the
-// cluster's T (<= CL) 128-channel weight tiles; the clusters share the tiles
-// out evenly (T and T-1 tiles).  A CTA reads only its K range of X, so the
-// outlier flags of those columns are final at once (all M rows of a column
-// are in the same CTA), quantises only those columns, and shares with its
-// peers just the flag words and the row maxima (one exchange of asynchronous
-// stores into the peers' shared memory, which complete on the receiver's
-// mbarrier).  The int32 partial sums of a tile go the same way to the tile's
-// owner (CTA j owns tile j) as soon as that tile's MMAs are complete, one slot
-// per peer, and the owner adds them to its own (exact in any order).
+// when that is fewer) split K: CTA r of a cluster owns the
+// r-th K range of the cluster's T (<= CL) 128-channel weight tiles.  It reads
+// only its K range of X, so the outlier flags of those columns are final at
+// once (all M rows of a column are in the same CTA), quantises only those
+// columns, and shares with its peers just the flag words and the row maxima
+// (one exchange of asynchronous stores into the peers' shared memory, which
+// complete on the receiver's mbarrier).  The int32 partial sums of a tile go
+// the same way to the tile's owner (CTA j owns tile j), one slot per source
+// CTA, and the owner adds the slots (exact in any order).
 //
-// Two shapes of the same kernel:
-//   256 threads, at most 113 KB of shared memory: two CTAs fit on one SM, so
-//     while a call runs (one CTA per SM), the next call on the stream already
-//     has its CTAs resident and streaming weights into their rings, waiting
-//     only for its X (programmatic dependent launch), and the call after it
-//     takes the SMs this call leaves;
-//   384 threads and up to 227 KB (one CTA per SM), for K ranges or
-//     shared-memory plans the small shape cannot hold.
-//
-// Warp roles:
+// Warp roles (384 threads):
 //   warp 0: TMA producer of 128 (channels) x 128 (K) int8 weight boxes;
 //   warp 1: tcgen05.mma kind::i8 with the weight as the 128-row A operand and
 //     the (padded) activation rows as the 16-column B operand ("swap AB"),
-//     one s32 TMEM accumulator per tile, a commit per finished tile;
-//   warps 2..: (a) outlier columns and row absmax of the CTA's K range, then
+//     one s32 TMEM accumulator per tile;
+//   warps 2-11: (a) outlier columns and row absmax of the CTA's K range, then
 //     (b) the int8 codes straight into shared memory in the tensor-core
 //     operand layout (128-byte rows, 128-byte swizzle, 8-row groups);
 //   warps 4-7 (after the X-side steps): the fp16 outlier product (d) of the
-//     owned tile while the weights stream, the hand-off of each finished
-//     tile's partial sums, then Y = fp16(acc * ra * ca / 127^2 + o).
+//     owned tile while the weights stream, then the reduction of the partial
+//     sums and Y = fp16(acc * ra * ca / 127^2 + o).
 #pragma once
 
 #include <cuda.h>
@@ -68,17 +58,16 @@ struct DecodeParams {
     uint64_t wait_limit_ns;
     uint32_t test_flags;        // bit 0: never signal that Xq is ready (timeout test)
     int num_tiles, kb_total;    // 128-channel tiles, 128-column K blocks
-    int num_clusters;           // cluster c owns tiles [c * num_tiles / num_clusters, (c + 1) * ...)
-    int cluster, stages, groups;  // groups = ceil(M / 8)
-    uint32_t tmem_cols;         // 32 columns per tile of the largest tile range, a power of two >= 32
+    int cluster, tiles_per_cluster, stages, groups;  // groups = ceil(M / 8)
     uint32_t off_xq, off_mask, off_pre, off_list, off_xo, off_oslot, off_red, off_bars;  // shared-memory offsets
 };
 
-constexpr int kDecSmemOutliers = 64;         // outlier columns whose x values are staged in shared memory
+constexpr int kDecThreads = 384;             // warp 0 TMA, warp 1 MMA, warps 2..11 X-side, 4..7 epilogue
+constexpr int kDecPro = kDecThreads - 64;    // threads of the X-side steps
+constexpr int kDecSmemOutliers = 128;        // outlier columns whose x values are staged in shared memory
 constexpr int kDecTileN = 128;
 constexpr int kDecStageBytes = kDecTileN * 128;  // 16 KB
 constexpr int kDecMaxCluster = 8;
-constexpr int kDecMaxTiles = 8;              // tiles per cluster (<= the cluster size)
 
 __device__ __forceinline__ float dec_half_to_float(uint32_t bits16) {
     return __half2float(__ushort_as_half((unsigned short)bits16));
@@ -128,16 +117,6 @@ __device__ __forceinline__ uint2 dec_quant8(uint4 v, uint32_t fl, float scale) {
     return make_uint2(lo, hi);
 }
 
-// 16-byte read-only load as a volatile instruction: issued once and kept in
-// registers (the compiler may neither repeat nor sink it).
-__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
-    uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
 // Pass (a) works on packed fp16 pairs with the native half2 compare and max:
 // |x| is the bit pattern with the sign cleared, __hge2_mask gives false for
 // NaN (so NaN is never an outlier) and __hmax2 returns the other operand when
@@ -185,37 +164,33 @@ __device__ __forceinline__ __half2 inlier_max8(uint4 a, uint32_t fl) {
 }
 
 // kR: rows per 8-column chunk group (8 or 16, >= M); kP: (chunk, row) pairs
-// per X-side thread (the CTA's K range has at most kP * (kThr - 64) / kR
-// chunks); kThr: threads (256: two CTAs per SM, 384: one).
-template <int kR, int kP, int kThr>
-__global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
+// per X-side thread (the CTA's K range has at most kP * kDecPro / kR chunks).
+template <int kR, int kP>
+__global__ void __launch_bounds__(kDecThreads, 1)
     k_decode_int8_sm100(const __grid_constant__ CUtensorMap tm_w, const DecodeParams p) {
-    constexpr int kPro = kThr - 64;  // threads of the X-side steps (warps 2..)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = smem;
     uint8_t* sxq = smem + p.off_xq;
     uint32_t* smask = reinterpret_cast<uint32_t*>(smem + p.off_mask);
     int* spre = reinterpret_cast<int*>(smem + p.off_pre);
-    uint16_t* slist = reinterpret_cast<uint16_t*>(smem + p.off_list);  // [kDecSmemOutliers] outlier columns
+    uint16_t* slist = reinterpret_cast<uint16_t*>(smem + p.off_list);
     uint16_t* sxo = reinterpret_cast<uint16_t*>(smem + p.off_xo);  // [kDecSmemOutliers][16] fp16 x values
     int* soslot = reinterpret_cast<int*>(smem + p.off_oslot);      // [kDecSmemOutliers] kept-row slot
-    uint32_t* sred = reinterpret_cast<uint32_t*>(smem + p.off_red);  // [CL-1][128][RS] peers' partial sums of the owned tile
+    uint32_t* sred = reinterpret_cast<uint32_t*>(smem + p.off_red);  // [CL][128][RS] partial sums of the owned tile
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bars);
     uint64_t* full = bars;
     uint64_t* empty = bars + p.stages;
-    uint64_t* tfull = bars + 2 * p.stages;   // [kDecMaxTiles]: tile j's MMAs are complete
-    uint64_t* xq_ready = tfull + kDecMaxTiles;
-    uint64_t* drain = xq_ready + 1;
-    uint64_t* xchg = xq_ready + 2;      // flag words and row maxima of every peer have arrived (tx bytes)
-    uint64_t* red_done = xq_ready + 3;  // every peer's partial sums have arrived (tx bytes)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xq_ready + 4);
+    uint64_t* tfull = bars + 2 * p.stages;
+    uint64_t* xq_ready = tfull + 1;
+    uint64_t* drain = tfull + 2;
+    uint64_t* xchg = tfull + 3;      // flag words and row maxima of every peer have arrived (tx bytes)
+    uint64_t* red_done = tfull + 4;  // every peer's partial sums have arrived (tx bytes)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 5);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     unsigned* sra_bits = reinterpret_cast<unsigned*>(tmem_slot + 2);  // [16] row absmax (fp16 bits)
     int* sflag = reinterpret_cast<int*>(tmem_slot + 18);              // [1] total outliers
     float* srs = reinterpret_cast<float*>(tmem_slot + 20);            // [16] ra / 127^2
-    uint32_t* sown = tmem_slot + 36;                                  // [16] this CTA's row maxima
-    uint32_t* swmax = tmem_slot + 52;                                 // [10][16] per-warp row maxima
     const uint16_t* __restrict__ Xg = p.X;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -230,14 +205,14 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
     // tile tile0 + rank when rank < nt
     const int rank = (int)cluster_ctarank();
     const int cid = blockIdx.x / CL;
-    const int tile0 = (int)((long long)cid * p.num_tiles / p.num_clusters);
-    const int nt = (int)((long long)(cid + 1) * p.num_tiles / p.num_clusters) - tile0;
+    const int tile0 = cid * p.tiles_per_cluster;
+    const int nt = max(0, min(p.tiles_per_cluster, p.num_tiles - tile0));
     const int kb_lo = p.kb_total * rank / CL;  // kb_total <= 1024, CL <= 8: no overflow
     const int kb_hi = p.kb_total * (rank + 1) / CL;
     const int c0 = kb_lo * 16, c1 = min(nchunk, kb_hi * 16);
     const bool owner = rank < nt;
     const bool has_acc = nt > 0 && kb_hi > kb_lo;
-    const uint32_t tmem_cols = p.tmem_cols;
+    const uint32_t tmem_cols = p.tiles_per_cluster <= 1 ? 32u : (p.tiles_per_cluster <= 2 ? 64u : (p.tiles_per_cluster <= 4 ? 128u : 256u));
 
     // Set-up is split by role so that the X-side steps, which gate the first
     // MMA, start at once: warp 0 initialises the mbarriers and starts the
@@ -255,7 +230,7 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
                 mbar_init(&full[s], 1);
                 mbar_init(&empty[s], 1);
             }
-            for (int j = 0; j < kDecMaxTiles; ++j) mbar_init(&tfull[j], 1);
+            mbar_init(tfull, 1);
             mbar_init(xq_ready, 1);
             mbar_init(drain, 1);
             mbar_init(xchg, 1);
@@ -264,7 +239,7 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
             fence_mbar_init();
             prefetch_tmap(&tm_w);
             // bytes the peers will store: their flag words and M row maxima
-            // each, and (owner) one partial-sum slot per peer
+            // each, and (owner) one partial-sum slot per CTA of the cluster
             uint32_t xb = 0;
             for (int q = 0; q < CL; ++q) {
                 if (q == rank) continue;
@@ -273,19 +248,17 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
             }
             if (xb) mbar_arrive_expect_tx(xchg, xb);
             else mbar_arrive(xchg);
-            const uint32_t rb = (uint32_t)((CL - 1) * kDecTileN * RS * 4);
-            if (owner && has_acc && rb) mbar_arrive_expect_tx(red_done, rb);
-            else mbar_arrive(red_done);
+            if (owner && has_acc) mbar_arrive_expect_tx(red_done, (uint32_t)(CL * kDecTileN * RS * 4));
         }
         __syncwarp();
         cluster_arrive();
-        named_bar_arrive(2, kThr);
+        named_bar_arrive(2, kDecThreads);
     } else if (warp == 1) {
         tmem_alloc(tmem_slot, tmem_cols);
         tmem_relinquish();
         tc_fence_before();
         cluster_arrive();
-        named_bar_sync(2, kThr);
+        named_bar_sync(2, kDecThreads);
         tc_fence_after();
         tmem_base = *tmem_slot;
     }
@@ -353,36 +326,37 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
                         da = da0;
                     }
                 }
-                if (ok) tc_commit(&tfull[j]);  // tile j's sums can leave while tile j+1 streams
             }
+
+            if (ok) tc_commit(tfull);
             if (issued) {
                 tc_commit(drain);
                 wait_drain(drain, 0, 50ull * 1000 * 1000);
             }
         }
     } else {
-        // ------------------------------------------------ X-side steps (warps 2..)
-        const int pt = threadIdx.x - 64;  // 0 .. kPro-1
+        // ------------------------------------------------ X-side steps (warps 2..11)
+        const int pt = threadIdx.x - 64;  // 0 .. kDecPro-1
         if (pt < 16) sra_bits[pt] = 0u;
-        for (int w = pt; w < nw; w += kPro) smask[w] = 0u;
-        named_bar_sync(1, kPro);
+        for (int w = pt; w < nw; w += kDecPro) smask[w] = 0u;
+        named_bar_sync(1, kDecPro);
         cluster_arrive();
         pdl_wait();  // X belongs to earlier work on the stream
         // (a) Thread pairs (8-column chunk, row): the kR rows of a chunk sit in
         // kR consecutive lanes, so a chunk's outlier flags are the OR of its
         // lanes' flags (shuffles), and a thread's row is the same for all its
-        // pairs (kPro is a multiple of 32 and of kR), so one running max
+        // pairs (kDecPro is a multiple of 32 and of kR), so one running max
         // and one scale per thread.  The values stay in registers for (b).
         const int prow = lane % kR;
         const bool row_ok = prow < M;
         // iterations that hold any pair of this CTA (the same for every thread)
-        const int nit = ((c1 - c0) * kR + kPro - 1) / kPro;
+        const int nit = ((c1 - c0) * kR + kDecPro - 1) / kDecPro;
         uint4 xv[kP];
         uint32_t cfl[kP];
 #pragma unroll
         for (int i = 0; i < kP; ++i) {
-            const int c = c0 + (pt + i * kPro) / kR;
-            if (i < nit && row_ok && c < c1) xv[i] = ld_nc_v4(reinterpret_cast<const uint4*>(Xg + (size_t)prow * K) + c);
+            const int c = c0 + (pt + i * kDecPro) / kR;
+            if (i < nit && row_ok && c < c1) xv[i] = __ldg(reinterpret_cast<const uint4*>(Xg + (size_t)prow * K) + c);
         }
         {
             // in phases over the iterations, so that their dependency chains
@@ -391,7 +365,7 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
             __half2 rmax2 = as_h2(0u);
 #pragma unroll
             for (int i = 0; i < kP; ++i) {
-                const int c = c0 + (pt + i * kPro) / kR;
+                const int c = c0 + (pt + i * kDecPro) / kR;
                 cfl[i] = (i < nit && row_ok && c < c1) ? flags8(abs8(xv[i]), thr2) : 0u;
             }
 #pragma unroll
@@ -400,58 +374,38 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
                 for (int i = 0; i < kP; ++i)
                     if (i < nit) cfl[i] |= __shfl_xor_sync(0xffffffffu, cfl[i], off);
             }
-            // A warp's lanes hold 32 / kR consecutive chunks of one iteration,
-            // starting at a multiple of 32 / kR (c0, kPro and the warp's first
-            // pair are multiples of 32): with kR = 8 that is one whole flag word,
-            // which lane 0 stores; with kR = 16, half a word (two warps OR it).
 #pragma unroll
             for (int i = 0; i < kP; ++i) {
-                if (i >= nit) continue;
-                const int c = c0 + (pt + i * kPro) / kR;
-                uint32_t word = (c < c1 ? cfl[i] : 0u) << ((lane / kR) * 8);
-#pragma unroll
-                for (int off = kR; off < 32; off <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, off);
-                const int cw = c - lane / kR;  // the warp's first chunk
-                if (lane == 0 && cw < c1) {
-                    if (kR == 8) smask[cw >> 2] = word << ((cw & 3) * 8);
-                    else if (word) atomicOr(&smask[cw >> 2], word << ((cw & 3) * 8));
+                const int c = c0 + (pt + i * kDecPro) / kR;
+                if (i < nit && c < c1) {
+                    if (prow == 0 && cfl[i]) atomicOr(&smask[c >> 2], cfl[i] << ((c & 3) * 8));
+                    if (row_ok) rmax2 = __hmax2(rmax2, inlier_max8(abs8(xv[i]), cfl[i]));
                 }
-                if (row_ok && c < c1) rmax2 = __hmax2(rmax2, inlier_max8(abs8(xv[i]), cfl[i]));
             }
             // non-negative fp16 bit patterns order like their values
             const uint32_t rb = as_u32(rmax2);
             uint32_t rmax = max(rb & 0xFFFFu, rb >> 16);
 #pragma unroll
             for (int off = kR; off < 32; off <<= 1) rmax = max(rmax, __shfl_xor_sync(0xffffffffu, rmax, off));
-            if (lane < kR) swmax[(warp - 2) * 16 + lane] = row_ok ? rmax : 0u;
+            if (lane < kR && row_ok && rmax) atomicMax(&sra_bits[prow], rmax);
         }
         // every X-side thread's flags and maxima are in; the mbarriers are
         // initialised and TMEM is allocated
-        named_bar_sync(2, kThr);
+        named_bar_sync(2, kDecThreads);
         tc_fence_after();
         tmem_base = *tmem_slot;
-        // this CTA's row maxima from the warps' partial maxima; atomically,
-        // because a peer's maximum may already have landed in sra_bits
-        if (pt >= kPro - 16 && pt - (kPro - 16) < M) {
-            const int m = pt - (kPro - 16);
-            uint32_t v = 0u;
-#pragma unroll
-            for (int w = 0; w < kPro / 32; ++w) v = max(v, swmax[w * 16 + (m % kR)]);
-            if (v) atomicMax(&sra_bits[m], v);
-            sown[m] = v;
-        }
         // this CTA's flag words (its K range covers whole words) and row
         // maxima to every peer; the peers' arrive the same way
         if (CL > 1) {
             cluster_wait();  // every peer's barriers and buffers are initialised
-            for (int w = c0 / 4 + pt; w < (c1 + 3) / 4; w += kPro) {
+            for (int w = c0 / 4 + pt; w < (c1 + 3) / 4; w += kDecPro) {
                 const uint32_t val = smask[w];
                 for (int q = 0; q < CL; ++q)
                     if (q != rank) st_async_u32(map_to_rank(&smask[w], (uint32_t)q), val, map_to_rank(xchg, (uint32_t)q));
             }
-            if (pt >= kPro - 16 && pt - (kPro - 16) < M) {
-                const int m = pt - (kPro - 16);
-                const uint32_t val = sown[m];  // this CTA's own maximum
+            if (pt >= kDecPro - 16 && pt - (kDecPro - 16) < M) {
+                const int m = pt - (kDecPro - 16);
+                const uint32_t val = sra_bits[m];
                 for (int q = 0; q < CL; ++q)
                     if (q != rank)
                         red_async_max_u32(map_to_rank(&sra_bits[m], (uint32_t)q), val, map_to_rank(xchg, (uint32_t)q));
@@ -468,7 +422,7 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
             const float scl = rmax > 0.0f ? __fdiv_rn(127.0f, rmax) : 0.0f;
 #pragma unroll
             for (int i = 0; i < kP; ++i) {
-                const int c = c0 + (pt + i * kPro) / kR;
+                const int c = c0 + (pt + i * kDecPro) / kR;
                 if (i < nit && row_ok && c < c1) {
                     const uint2 q = dec_quant8(xv[i], cfl[i], scl);
                     *reinterpret_cast<uint2*>(sxq + dec_xq_off(prow, (c - c0) * 8, p.groups)) = q;
@@ -482,7 +436,7 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
             if (blockIdx.x == 0 && lane < M) p.ra_out[lane] = rmax;
         }
         fence_proxy_async_smem();
-        named_bar_sync(1, kPro);
+        named_bar_sync(1, kDecPro);
         if (pt == 0 && !(p.test_flags & 1u)) mbar_arrive(xq_ready);
         // slot prefix of the outlier flags (off the critical path of the codes)
         if (warp == 2) {
@@ -502,23 +456,25 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
             }
             if (lane == 0) sflag[0] = carry;
         }
-        named_bar_sync(1, kPro);
+        named_bar_sync(1, kDecPro);
         const int total = sflag[0];
         const int n_eff = min(total, p.cap);
-        // x values and kept-row slots of the first kDecSmemOutliers outliers
-        // into shared memory; CTA 0 publishes the ascending list
-        for (int w = pt; w < nw; w += kPro) {
+        // outlier list (ascending) into shared memory with the x values and
+        // kept-row slots of the first kDecSmemOutliers; CTA 0 publishes it
+        for (int w = pt; w < nw; w += kDecPro) {
             uint32_t word = smask[w];
             int s = spre[w];
-            while (word && s < n_eff) {
+            while (word) {
                 const int b = __ffs(word) - 1;
                 const int k = w * 32 + b;
-                if (blockIdx.x == 0) p.idx_out[s] = k;
-                if (s < kDecSmemOutliers) {
+                if (s < n_eff) {
                     slist[s] = (uint16_t)k;
-                    soslot[s] = p.keep_slot[k];
+                    if (blockIdx.x == 0) p.idx_out[s] = k;
+                    if (s < kDecSmemOutliers) {
+                        soslot[s] = p.keep_slot[k];
 #pragma unroll
-                    for (int m = 0; m < 16; ++m) sxo[s * 16 + m] = m < M ? Xg[(size_t)m * K + k] : (uint16_t)0;
+                        for (int m = 0; m < 16; ++m) sxo[s * 16 + m] = m < M ? Xg[(size_t)m * K + k] : (uint16_t)0;
+                    }
                 }
                 ++s;
                 word &= word - 1;
@@ -528,7 +484,7 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
             *p.n_out = total;
             if (total > p.cap) atomicOr(p.status, kStatusOverflow);
         }
-        named_bar_sync(1, kPro);
+        named_bar_sync(1, kDecPro);
 
         if (warp >= 4 && warp < 8) {
             // ------------------------------------------------ epilogue (warps 4..7)
@@ -537,101 +493,66 @@ __global__ void __launch_bounds__(kThr, kThr <= 256 ? 2 : 1)
             const int n = (tile0 + rank) * kDecTileN + ch;
             // (d) fp16 outlier product of the owned tile, ascending j, while the
             // weights stream: the weight value of outlier j is the kept fp16 row
-            // or the dequantised int8 row; the outliers are the set bits of the
-            // flag words in order
+            // or the dequantised int8 row
             float o[16];
 #pragma unroll
             for (int m = 0; m < 16; ++m) o[m] = 0.0f;
             const float cav = (owner && n < N) ? p.ca[n] : 0.0f;
-            if (owner && n < N && n_eff > 0) {
-                // the staged outliers, eight at a time: their eight weight
-                // loads are independent and in flight together
+            if (owner && n < N) {
                 const int n_fast = min(n_eff, kDecSmemOutliers);
-                for (int j0 = 0; j0 < n_fast; j0 += 8) {
-                    float wv[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int j = j0 + u;
-                        wv[u] = 0.0f;
-                        if (j < n_fast) {
-                            const int slot = soslot[j];
-                            if (slot >= 0) {
-                                wv[u] = dec_half_to_float(p.w_keep[(size_t)slot * N + n]);
-                            } else {
-                                const float tq = __fmul_rn((float)p.wq[(size_t)n * K + slist[j]], cav);
-                                wv[u] = __half2float(__float2half_rn(__fdiv_rn(tq, 127.0f)));
-                            }
-                        }
+#pragma unroll 4
+                for (int j = 0; j < n_fast; ++j) {
+                    const int slot = soslot[j];
+                    float w;
+                    if (slot >= 0) {
+                        w = dec_half_to_float(p.w_keep[(size_t)slot * N + n]);
+                    } else {
+                        const float tq = __fmul_rn((float)p.wq[(size_t)n * K + slist[j]], cav);
+                        w = __half2float(__float2half_rn(__fdiv_rn(tq, 127.0f)));
                     }
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        if (j0 + u < n_fast) {
-#pragma unroll
-                            for (int m = 0; m < 16; ++m)
-                                if (m < M) o[m] = fmaf(dec_half_to_float(sxo[(j0 + u) * 16 + m]), wv[u], o[m]);
-                        }
-                    }
+                    for (int m = 0; m < 16; ++m)
+                        if (m < M) o[m] = fmaf(dec_half_to_float(sxo[j * 16 + m]), w, o[m]);
                 }
-                // the rest (more outlier columns than are staged): in order,
-                // from the flag words
-                if (n_eff > n_fast) {
-                    int j = 0;
-                    for (int w = 0; w < nw && j < n_eff; ++w) {
-                        uint32_t word = smask[w];
-                        while (word && j < n_eff) {
-                            const int k = w * 32 + __ffs(word) - 1;
-                            word &= word - 1;
-                            if (j++ < n_fast) continue;
-                            const int slot = p.keep_slot[k];
-                            float wv;
-                            if (slot >= 0) {
-                                wv = dec_half_to_float(p.w_keep[(size_t)slot * N + n]);
-                            } else {
-                                const float tq = __fmul_rn((float)p.wq[(size_t)n * K + k], cav);
-                                wv = __half2float(__float2half_rn(__fdiv_rn(tq, 127.0f)));
-                            }
-#pragma unroll
-                            for (int m = 0; m < 16; ++m)
-                                if (m < M) o[m] = fmaf(dec_half_to_float(Xg[(size_t)m * K + k]), wv, o[m]);
-                        }
+                for (int j = n_fast; j < n_eff; ++j) {
+                    const int k = slist[j];
+                    const int slot = p.keep_slot[k];
+                    float w;
+                    if (slot >= 0) {
+                        w = dec_half_to_float(p.w_keep[(size_t)slot * N + n]);
+                    } else {
+                        const float tq = __fmul_rn((float)p.wq[(size_t)n * K + k], cav);
+                        w = __half2float(__float2half_rn(__fdiv_rn(tq, 127.0f)));
                     }
+#pragma unroll
+                    for (int m = 0; m < 16; ++m)
+                        if (m < M) o[m] = fmaf(dec_half_to_float(Xg[(size_t)m * K + k]), w, o[m]);
                 }
             }
-            // partial sums of each tile, as soon as its MMAs are complete, into
-            // this CTA's slot of the tile owner's buffer (16-byte asynchronous
-            // stores, the rows of one channel together), completing on the
-            // owner's barrier; the owner keeps its own in registers
-            uint32_t own[16];
-#pragma unroll
-            for (int m = 0; m < 16; ++m) own[m] = 0u;
-            bool got = has_acc;
-            for (int j = 0; got && j < nt; ++j) {
-                got = __all_sync(0xffffffffu, wait_bounded_sleep(&tfull[j], 0, wctx));
-                if (!got) break;
+            // partial sums of every tile of this CTA into this CTA's slot of the
+            // tile owner's buffer (16-byte asynchronous stores, rows of one
+            // channel together), completing on the owner's barrier
+            if (has_acc && __all_sync(0xffffffffu, wait_bounded_sleep(tfull, 0, wctx))) {
                 tc_fence_after();
-                uint32_t r[16];
-                tmem_ld16(tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(32 * j), r);
-                tmem_wait_ld();
-                if (j == rank) {
-#pragma unroll
-                    for (int m = 0; m < 16; ++m) own[m] = r[m];
-                    continue;
-                }
-                const int slot = rank < j ? rank : rank - 1;
-                const uint32_t dst = map_to_rank(&sred[(size_t)(slot * kDecTileN + ch) * RS], (uint32_t)j);
-                const uint32_t mb = map_to_rank(red_done, (uint32_t)j);
-                st_async_v4(dst, r[0], r[1], r[2], r[3], mb);
-                st_async_v4(dst + 16, r[4], r[5], r[6], r[7], mb);
-                if (RS == 16) {
-                    st_async_v4(dst + 32, r[8], r[9], r[10], r[11], mb);
-                    st_async_v4(dst + 48, r[12], r[13], r[14], r[15], mb);
+                for (int j = 0; j < nt; ++j) {
+                    uint32_t r[16];
+                    tmem_ld16(tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(32 * j), r);
+                    tmem_wait_ld();
+                    const uint32_t dst = map_to_rank(&sred[(size_t)(rank * kDecTileN + ch) * RS], (uint32_t)j);
+                    const uint32_t mb = map_to_rank(red_done, (uint32_t)j);
+                    st_async_v4(dst, r[0], r[1], r[2], r[3], mb);
+                    st_async_v4(dst + 16, r[4], r[5], r[6], r[7], mb);
+                    if (RS == 16) {
+                        st_async_v4(dst + 32, r[8], r[9], r[10], r[11], mb);
+                        st_async_v4(dst + 48, r[12], r[13], r[14], r[15], mb);
+                    }
                 }
             }
-            if (owner && got && __all_sync(0xffffffffu, wait_bounded_sleep(red_done, 0, wctx)) && n < N) {
+            if (owner && has_acc && __all_sync(0xffffffffu, wait_bounded_sleep(red_done, 0, wctx)) && n < N) {
                 uint32_t sum[16];
 #pragma unroll
-                for (int m = 0; m < 16; ++m) sum[m] = own[m];
-                for (int q = 0; q < CL - 1; ++q) {
+                for (int m = 0; m < 16; ++m) sum[m] = 0u;
+                for (int q = 0; q < CL; ++q) {
                     const uint4* src = reinterpret_cast<const uint4*>(&sred[(size_t)(q * kDecTileN + ch) * RS]);
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {

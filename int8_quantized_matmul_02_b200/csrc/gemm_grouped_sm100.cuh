@@ -8,18 +8,20 @@
 // product.
 //
 //   acc_g[m, n] = sum_{k in group g} Xq[m, k] * Wq[n, k]    tcgen05 kind::i8, s32 in TMEM
-//   v[m, n]     = sum_g ((float(acc_g) * ra[m,g]) * ca[g,n]) / 127^2   fp32, ascending g
+//   v[m, n]     = sum_g acc_g * (ra[m,g] / 127^2) * ca[g,n]  fp32, ascending g
 //   v[m, n]    += sum_j Xo[m, j] * Wo[n, j]                 tcgen05 kind::f16 onto v in TMEM
 //   Y[m, n]     = fp16(v)
 //
 // The accumulation of a group ends in one of two s32 TMEM accumulators; while
 // the tensor cores fill the other with the next group, the epilogue drains
-// it, applies the group's constants and adds the result to the running fp32
-// sum, which also lives in TMEM (columns 256-383).  The running sum uses the
-// same operations in the same order as the definition, so before the outlier
-// product it is exact to the bit.  The pair tile is 256 x 128 (each CTA 128
-// rows; each CTA stages its 128 rows of A and 64 rows of B per 128-byte K
-// slice), persistent CTA pairs walk the tiles in M-grouped order.
+// it, applies the group's constants (acc * (ra / 127^2) * ca, one multiply and
+// one fused multiply-add per element) and adds the result to the tile's
+// running fp32 sums, which each epilogue thread keeps in registers (its row,
+// 64 columns).  With outlier columns the sums go to TMEM (columns 256-383)
+// once per tile, and the fp16 outlier product accumulates onto them there.
+// The pair tile is 256 x 128 (each CTA 128 rows; each CTA stages its 128 rows
+// of A and 64 rows of B per 128-byte K slice); persistent CTA pairs walk the
+// tiles in M-grouped order.
 //   warp 0     TMA producer (completion counted on the even CTA's barrier);
 //   warp 1     TMEM allocation (pair-wide, 512 columns) and, in the even CTA,
 //              the MMA issuer;
@@ -52,7 +54,9 @@ constexpr int kGGBBytes = 64 * 128;                // this CTA's B rows
 constexpr int kGGStageBytes = kGGABytes + kGGBBytes;  // 24 KB
 constexpr int kGGEpiWarps = 8;
 constexpr int kGGThreads = 64 + 32 * kGGEpiWarps;  // 320
-constexpr int kGGSmemBytes = 1024 + kGGStages * kGGStageBytes + kGGEpiWarps * 2 * kGemmEpiBufBytes + 256;
+constexpr int kGGCaBytes = 2 * 64 * 4;            // per epilogue warp: two groups' 64 column constants
+constexpr int kGGSmemBytes =
+    1024 + kGGStages * kGGStageBytes + kGGEpiWarps * (2 * kGemmEpiBufBytes + kGGCaBytes) + 256;
 constexpr uint32_t kGGSumCol = 256;                // running fp32 sums; accumulators at 0 and 128
 
 template <bool kWriteAcc>
@@ -64,7 +68,8 @@ __global__ void __launch_bounds__(kGGThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = smem;
     uint8_t* epi = smem + kGGStages * kGGStageBytes;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(epi + kGGEpiWarps * 2 * kGemmEpiBufBytes);
+    float* scas = reinterpret_cast<float*>(epi + kGGEpiWarps * 2 * kGemmEpiBufBytes);  // [warps][2][64]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(epi + kGGEpiWarps * (2 * kGemmEpiBufBytes + kGGCaBytes));
     uint64_t* full = bars;                    // [stages] even CTA: both CTAs' bytes
     uint64_t* empty = bars + kGGStages;       // [stages] each CTA: its stage is free
     uint64_t* tfull = bars + 2 * kGGStages;   // [2] each CTA: a group's int8 sums are ready
@@ -236,6 +241,7 @@ __global__ void __launch_bounds__(kGGThreads, 1)
         const int ew = warp - 2;
         const int quad = warp & 3, half = ew >> 2;  // lane quadrant, 64-column half
         uint8_t* bufs = epi + ew * 2 * kGemmEpiBufBytes;
+        float* wca = scas + ew * 128;  // this warp's two slots of 64 column constants
         const uint32_t tempty_even[2] = {map_to_rank(&tempty[0], 0), map_to_rank(&tempty[1], 0)};
         const uint32_t tscaled_even = map_to_rank(tscaled, 0);
         int buf_i = 0;
@@ -250,6 +256,27 @@ __global__ void __launch_bounds__(kGGThreads, 1)
             const int colw = nb * kGGBN + half * 64;  // this warp's first column
             const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
             const uint32_t tsum = tmem_base + lane_off + kGGSumCol + (uint32_t)(half * 64);
+            // the tile's running sums of this thread's row and 64 columns stay
+            // in registers across the groups
+            float v[64];
+#pragma unroll
+            for (int i = 0; i < 64; ++i) v[i] = 0.0f;
+            // the group constants of this warp's 64 columns go to shared memory
+            // one group ahead (asynchronous 16-byte copies, lanes 0-15), the row
+            // constant one group ahead in a register
+            auto fetch_ca = [&](int g) {
+                if (lane < 16) {
+                    const int col = colw + 4 * lane;
+                    const float* src = gp.ca + (size_t)g * p.N + col;
+                    const uint32_t dst = smem_u32(wca + (g & 1) * 64 + 4 * lane);
+                    const int bytes = col < p.N ? 16 : 0;  // N % 16 == 0: a 4-column piece is in or out
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes)
+                                 : "memory");
+                }
+                asm volatile("cp.async.commit_group;" ::: "memory");
+            };
+            fetch_ca(0);
+            float ra_next = row < p.M ? gp.ra[(size_t)row * ng] : 0.0f;
             for (int g = 0; g < ng; ++g) {
                 if (!__all_sync(0xffffffffu, wait_bounded_cluster(&tfull[acc], acc_phase, wctx))) {
                     ok = false;
@@ -257,95 +284,78 @@ __global__ void __launch_bounds__(kGGThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t tacc = tmem_base + lane_off + (uint32_t)(acc * kGGBN + half * 64);
-                const float rg = row < p.M ? gp.ra[(size_t)row * ng + g] : 0.0f;
-                const bool last = g == ng - 1;
-#pragma unroll 1
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t r[32], sv[32];
-                    tmem_ld32(tacc + 32 * c, r);
-                    if (g > 0) tmem_ld32(tsum + 32 * c, sv);
-                    tmem_wait_ld();
-                    const int col = colw + 32 * c;
-                    if (kWriteAcc && row < p.M) {
-#pragma unroll 4
-                        for (int i = 0; i < 32; ++i)
-                            if (col + i < p.N) gp.acc_out[((size_t)row * p.N + col + i) * ng + g] = (int32_t)r[i];
-                    }
-                    float cav[32];
-                    load_ca32(gp.ca + (size_t)g * p.N, col, p.N, cav);
-                    float v[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        float t = __fmul_rn(__fmul_rn((float)(int32_t)r[i], rg), cav[i]);
-                        t = __fdiv_rn(t, 16129.0f);
-                        v[i] = __fadd_rn(g > 0 ? __uint_as_float(sv[i]) : 0.0f, t);
-                    }
-                    if (last && n_ob == 0) {
-                        // no outlier product: this is Y (v + 0 in the definition)
-                        uint8_t* buf = bufs + buf_i * kGemmEpiBufBytes;
-                        if (lane == 0) bulk_wait_read<1>();
-                        __syncwarp();
-                        float lo[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) lo[i] = __fadd_rn(v[i], 0.0f);
-                        stage_row32(buf, lane, c & 1, lo);
-                        if (c == 1) {
-                            fence_proxy_async_smem();
-                            __syncwarp();
-                            if (lane == 0) {
-                                if (colw < p.N && row0 < p.M) tma_store_2d(&tm_y, buf, colw, row0);
-                                bulk_commit();
-                            }
-                            buf_i ^= 1;
-                        }
-                    } else {
-                        uint32_t w[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(v[i]);
-                        tmem_st32(tsum + 32 * c, w);
-                    }
+                // ra / 127^2 once per row and group; each term is acc * (ra / 127^2) * ca
+                const float rs = __fmul_rn(ra_next, 1.0f / 16129.0f);
+                if (g + 1 < ng) {
+                    fetch_ca(g + 1);
+                    ra_next = row < p.M ? gp.ra[(size_t)row * ng + g + 1] : 0.0f;
+                } else {
+                    asm volatile("cp.async.commit_group;" ::: "memory");  // keeps the group count in step
                 }
-                tmem_wait_st();
+                uint32_t r[64];
+                tmem_ld32(tacc, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+                tmem_ld32(tacc + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+                tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive_cluster(tempty_even[acc]);                   // the accumulator is free
-                    if (last && n_ob > 0) mbar_arrive_cluster(tscaled_even);  // the sums are in TMEM
-                }
+                if (lane == 0) mbar_arrive_cluster(tempty_even[acc]);  // the accumulator is free
                 if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1;
                 }
+                if (kWriteAcc && row < p.M) {
+#pragma unroll 4
+                    for (int i = 0; i < 64; ++i)
+                        if (colw + i < p.N) gp.acc_out[((size_t)row * p.N + colw + i) * ng + g] = (int32_t)r[i];
+                }
+                asm volatile("cp.async.wait_group 1;" ::: "memory");  // this group's constants have landed
+                __syncwarp();
+                const float4* cs = reinterpret_cast<const float4*>(wca + (g & 1) * 64);
+#pragma unroll
+                for (int q4 = 0; q4 < 16; ++q4) {
+                    const float4 c4 = cs[q4];
+                    v[4 * q4 + 0] = fmaf(__fmul_rn((float)(int32_t)r[4 * q4 + 0], rs), c4.x, v[4 * q4 + 0]);
+                    v[4 * q4 + 1] = fmaf(__fmul_rn((float)(int32_t)r[4 * q4 + 1], rs), c4.y, v[4 * q4 + 1]);
+                    v[4 * q4 + 2] = fmaf(__fmul_rn((float)(int32_t)r[4 * q4 + 2], rs), c4.z, v[4 * q4 + 2]);
+                    v[4 * q4 + 3] = fmaf(__fmul_rn((float)(int32_t)r[4 * q4 + 3], rs), c4.w, v[4 * q4 + 3]);
+                }
+                __syncwarp();  // every lane has read the slot before it is refilled
             }
             if (!ok) break;
             if (n_ob > 0) {
+                // the outlier product accumulates onto the sums in TMEM
+                uint32_t w[64];
+#pragma unroll
+                for (int i = 0; i < 64; ++i) w[i] = __float_as_uint(v[i]);
+                tmem_st32(tsum, *reinterpret_cast<uint32_t(*)[32]>(&w[0]));
+                tmem_st32(tsum + 32, *reinterpret_cast<uint32_t(*)[32]>(&w[32]));
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(tscaled_even);
                 if (!__all_sync(0xffffffffu, wait_bounded_cluster(tfull2, tile_phase, wctx))) break;
                 tc_fence_after();
                 tile_phase ^= 1;
-                uint32_t r0[32], r1[32];
-                tmem_ld32(tsum, r0);
-                tmem_ld32(tsum + 32, r1);
+                tmem_ld32(tsum, *reinterpret_cast<uint32_t(*)[32]>(&w[0]));
+                tmem_ld32(tsum + 32, *reinterpret_cast<uint32_t(*)[32]>(&w[32]));
                 tmem_wait_ld();
-                float v0[32], v1[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    v0[i] = __uint_as_float(r0[i]);
-                    v1[i] = __uint_as_float(r1[i]);
-                }
-                uint8_t* buf = bufs + buf_i * kGemmEpiBufBytes;
-                if (lane == 0) bulk_wait_read<1>();
-                __syncwarp();
-                stage_row32(buf, lane, 0, v0);
-                stage_row32(buf, lane, 1, v1);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    if (colw < p.N && row0 < p.M) tma_store_2d(&tm_y, buf, colw, row0);
-                    bulk_commit();
-                }
-                buf_i ^= 1;
+                for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(w[i]);
             }
+            uint8_t* buf = bufs + buf_i * kGemmEpiBufBytes;
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+            stage_row32(buf, lane, 0, *reinterpret_cast<const float(*)[32]>(&v[0]));
+            stage_row32(buf, lane, 1, *reinterpret_cast<const float(*)[32]>(&v[32]));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                if (colw < p.N && row0 < p.M) tma_store_2d(&tm_y, buf, colw, row0);
+                bulk_commit();
+            }
+            buf_i ^= 1;
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");  // no copy into shared memory outlives the loop
         if (lane == 0) bulk_wait_all<0>();
         __syncwarp();
     }

@@ -29,9 +29,6 @@ constexpr int kVersion = 100;  // 0.1.0
 constexpr uint64_t kDefaultWaitNs = 2000ull * 1000 * 1000;
 constexpr int kMaxK = 131072;
 constexpr int kMaxSmemOptin = 232448;  // 227 KB per block on sm_100
-// Two CTAs of 113 KB (plus the 1 KB the hardware keeps per CTA) fit in the
-// 228 KB of shared memory of one SM.
-constexpr int kDecSmallSmem = 113 * 1024;
 constexpr int kMaxDecodeRows = 16;
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -75,13 +72,9 @@ int8mm_status current_device(int* dev_out, DeviceInfo** info_out) {
                                  kGemmSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(k_gemm_int8_sm100<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGemmSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(k_decode_int8_sm100<8, 8, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kDecSmallSmem) != cudaSuccess ||
-            cudaFuncSetAttribute(k_decode_int8_sm100<16, 16, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kDecSmallSmem) != cudaSuccess ||
-            cudaFuncSetAttribute(k_decode_int8_sm100<8, 8, 384>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(k_decode_int8_sm100<8, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kMaxSmemOptin) != cudaSuccess ||
-            cudaFuncSetAttribute(k_decode_int8_sm100<16, 16, 384>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(k_decode_int8_sm100<16, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kMaxSmemOptin) != cudaSuccess ||
             cudaFuncSetAttribute(k_gemm_int8_grouped<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGGSmemBytes) != cudaSuccess ||
@@ -125,7 +118,7 @@ int cluster_capacity(DeviceInfo* d, int cl) {
         cfg.attrs = a;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, k_decode_int8_sm100<8, 8, 384>, &cfg) != cudaSuccess || n <= 0) {
+        if (cudaOccupancyMaxActiveClusters(&n, k_decode_int8_sm100<8, 8>, &cfg) != cudaSuccess || n <= 0) {
             cudaGetLastError();
             n = std::max(1, d->sm_count / cl);
         }
@@ -306,65 +299,58 @@ uint32_t fp16_threshold_bits2(float thr) {
     return lo | (lo << 16);
 }
 
-// Plan of the decode kernel: its shape (256 threads with at most
-// kDecSmallSmem bytes of shared memory, so that two CTAs fit on one SM, or
-// 384 threads with up to 227 KB), clusters of `cluster` CTAs splitting K, the
-// number of clusters (tiles shared out evenly, at most `cluster` per
-// cluster), a TMA ring of `stages` 16 KB boxes, and the shared-memory offsets.
+// Plan of the decode kernel: clusters of `cluster` CTAs split K (each CTA
+// one K range of the cluster's `tiles` 128-channel tiles), a TMA ring of
+// `stages` 16 KB boxes, and the shared-memory offsets.
 struct DecodePlan {
-    int threads, cluster, clusters, max_tiles, stages, groups, grid, mr;  // mr: rows per chunk group (8 or 16)
-    uint32_t tmem_cols;
+    int cluster, tiles, stages, groups, grid, mr;  // mr: rows per chunk group (8 or 16)
     uint32_t off_xq, off_mask, off_pre, off_list, off_xo, off_oslot, off_red, off_bars, bytes;
 };
 
-// (chunk, row) pairs each X-side thread holds in registers (template kP of
-// the kernel): rows per chunk group 8 -> 8 pairs, 16 -> 16 pairs.
-constexpr int decode_pairs(int mr) { return mr == 8 ? 8 : 16; }
-
-// dev == nullptr: no device limit on the number of clusters (only asks
-// whether the shape fits the kernel at all).
-bool decode_plan_shape(int M, int K, int N, DeviceInfo* dev, int threads, size_t smem_cap, int min_stages,
-                       DecodePlan* P) {
+// False when (M, K, cap) does not fit the kernel: M > 16, a CTA's K range
+// wider than its X-side threads hold in registers, or shared memory.
+bool decode_plan(int M, int K, int N, int cap, int sms, DecodePlan* P) {
+    if (M < 1 || M > kMaxDecodeRows) return false;
     const int kbt = cdiv(K, 128);
-    const int mr = M <= 8 ? 8 : 16;
-    const int chunks_max = decode_pairs(mr) * (threads - 64) / mr;  // 8-column chunks of X one CTA holds
+    // a CTA's K range holds at most kDecPro 8-column chunks (kP * kDecPro / kR)
+    int cl = 0;
+    for (int c : {4, 8}) {
+        const int cc = std::min(c, kbt);
+        if (cdiv(kbt, cc) * 16 <= kDecPro) {
+            cl = cc;
+            break;
+        }
+    }
+    if (cl == 0) return false;
     const int tiles = cdiv(N, kDecTileN);
+    // fewest tiles per cluster that keep the grid within one wave
+    int t = cl;
+    for (int c = 1; c <= cl; ++c) {
+        if ((long long)cl * cdiv(tiles, c) <= sms) {
+            t = c;
+            break;
+        }
+    }
     const int groups = (M + 7) / 8;
     const int nw = cdiv(K, 32);
-    for (int c : {4, 8}) {
-        const int cl = std::min(c, kbt);
-        if (cdiv(kbt, cl) * 16 > chunks_max) continue;
-        // clusters: one CTA per SM in one wave when the tiles allow (at most
-        // cl tiles per cluster), else as many waves as needed with cl tiles
-        // per cluster
-        const int cap = dev ? cluster_capacity(dev, cl) : (1 << 20);
-        int ncl = std::max(1, std::min(tiles, cap));
-        if (cdiv(tiles, ncl) > cl) ncl = cdiv(tiles, cl);
-        const int tmax = cdiv(tiles, ncl);
-        uint32_t tcols = 32;
-        while (tcols < (uint32_t)(32 * tmax)) tcols *= 2;
-        const size_t xq = (size_t)(cdiv(kbt, cl) * groups + 1) * 1024;
-        const size_t mask = align_up((size_t)nw * 4, 16);
-        const size_t pre = align_up((size_t)nw * 4, 16);
-        const size_t list = (size_t)kDecSmemOutliers * 2;
-        const size_t xo = (size_t)kDecSmemOutliers * 16 * 2;
-        const size_t oslot = (size_t)kDecSmemOutliers * 4;
-        const size_t red = (size_t)(cl - 1) * kDecTileN * 8 * groups * 4;  // one partial-sum slot per peer
-        const size_t fixed = xq + mask + pre + list + xo + oslot + red;
-        for (int s = 16; s >= min_stages; --s) {
-            // + TMEM address, abort flag, row maxima, count, scales, own and per-warp row maxima
-            const size_t bars = (size_t)(2 * s + kDecMaxTiles + 4) * 8 + 1024;
-            const size_t total = 1024 + (size_t)s * kDecStageBytes + fixed + bars;
-            if (total > smem_cap) continue;
-            P->threads = threads;
+    const size_t xq = (size_t)(cdiv(kbt, cl) * groups + 1) * 1024;
+    const size_t mask = align_up((size_t)nw * 4, 16);
+    const size_t pre = align_up((size_t)nw * 4, 16);
+    const size_t list = align_up((size_t)std::min(K, std::max(cap, 1)) * 2, 16);
+    const size_t xo = (size_t)kDecSmemOutliers * 16 * 2;
+    const size_t oslot = (size_t)kDecSmemOutliers * 4;
+    const size_t red = (size_t)cl * kDecTileN * 8 * groups * 4;  // one partial-sum slot per CTA of the cluster
+    const size_t fixed = xq + mask + pre + list + xo + oslot + red;
+    for (int s = 16; s >= 4; --s) {
+        const size_t bars = (size_t)(2 * s + 5) * 8 + 256;
+        const size_t total = 1024 + (size_t)s * kDecStageBytes + fixed + bars;
+        if (total <= (size_t)kMaxSmemOptin) {
             P->cluster = cl;
-            P->clusters = ncl;
-            P->max_tiles = tmax;
+            P->tiles = t;
             P->stages = s;
             P->groups = groups;
-            P->grid = cl * ncl;
-            P->mr = mr;
-            P->tmem_cols = tcols;
+            P->grid = cl * cdiv(tiles, t);
+            P->mr = M <= 8 ? 8 : 16;
             size_t o = (size_t)s * kDecStageBytes;
             P->off_xq = (uint32_t)o;
             o += xq;
@@ -388,14 +374,6 @@ bool decode_plan_shape(int M, int K, int N, DeviceInfo* dev, int threads, size_t
     return false;
 }
 
-// False when (M, K) does not fit the kernel: M > 16, or a CTA's K range wider
-// than its X-side threads hold in registers even in clusters of 8.
-bool decode_plan(int M, int K, int N, DeviceInfo* dev, DecodePlan* P) {
-    if (M < 1 || M > kMaxDecodeRows) return false;
-    return decode_plan_shape(M, K, N, dev, 256, kDecSmallSmem, 4, P) ||
-           decode_plan_shape(M, K, N, dev, 384, kMaxSmemOptin, 4, P);
-}
-
 // Parameters of one decode launch (the workspace pointers are the caller's).
 DecodeParams decode_params(const uint16_t* X, int M, const int8mm_weight* w, float threshold, int cap, uint16_t* Y,
                            const DecodePlan& dp) {
@@ -413,11 +391,10 @@ DecodeParams decode_params(const uint16_t* X, int M, const int8mm_weight* w, flo
     p.Y = Y;
     p.num_tiles = cdiv(w->N, kDecTileN);
     p.kb_total = cdiv(w->K, 128);
-    p.num_clusters = dp.clusters;
     p.cluster = dp.cluster;
+    p.tiles_per_cluster = dp.tiles;
     p.stages = dp.stages;
     p.groups = dp.groups;
-    p.tmem_cols = dp.tmem_cols;
     p.off_xq = dp.off_xq;
     p.off_mask = dp.off_mask;
     p.off_pre = dp.off_pre;
@@ -431,15 +408,9 @@ DecodeParams decode_params(const uint16_t* X, int M, const int8mm_weight* w, flo
 
 cudaError_t launch_decode(const DecodePlan& dp, const CUtensorMap& tm_w, const DecodeParams& p, cudaStream_t s,
                           bool pdl) {
-    const dim3 grid(dp.grid), block(dp.threads);
-    if (dp.threads == 256) {
-        if (dp.mr == 8)
-            return launch_ex(k_decode_int8_sm100<8, decode_pairs(8), 256>, grid, block, dp.bytes, s, pdl, dp.cluster, tm_w, p);
-        return launch_ex(k_decode_int8_sm100<16, decode_pairs(16), 256>, grid, block, dp.bytes, s, pdl, dp.cluster, tm_w, p);
-    }
     if (dp.mr == 8)
-        return launch_ex(k_decode_int8_sm100<8, decode_pairs(8), 384>, grid, block, dp.bytes, s, pdl, dp.cluster, tm_w, p);
-    return launch_ex(k_decode_int8_sm100<16, decode_pairs(16), 384>, grid, block, dp.bytes, s, pdl, dp.cluster, tm_w, p);
+        return launch_ex(k_decode_int8_sm100<8, 8>, dim3(dp.grid), dim3(kDecThreads), dp.bytes, s, pdl, dp.cluster, tm_w, p);
+    return launch_ex(k_decode_int8_sm100<16, 16>, dim3(dp.grid), dim3(kDecThreads), dp.bytes, s, pdl, dp.cluster, tm_w, p);
 }
 
 // ------------------------------------------------------------------ 4-bit weight-only decode
@@ -465,8 +436,8 @@ bool int4_shape_ok(int K, int N, int G) {
 }
 
 // Plan of the 4-bit kernel: clusters of `cluster` CTAs split K in 256-k
-// boxes, tiles shared out as in the 8-bit decode plan; two CTAs per SM when
-// the plan fits in kDecSmallSmem.
+// boxes, tiles shared out evenly (at most `cluster` per cluster), one CTA per
+// SM (the kernel takes the whole TMEM), one wave when the tiles allow.
 struct Int4Plan {
     int cluster, clusters, stages, xrows, grid;
     uint32_t tmem_cols, off_x, off_red, off_bars, bytes;
@@ -702,7 +673,7 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
 
     // whether the decode kernel fits does not depend on the device; its grid does
     DecodePlan dp{};
-    const bool decode_fits = decode_plan(M, K, N, nullptr, &dp);
+    const bool decode_fits = decode_plan(M, K, N, max_outliers, 1 << 20, &dp);
     bool use_decode;
     if (path == INT8MM_PATH_DECODE) {
         if (!decode_fits) return INT8MM_ERR_INVALID_ARGUMENT;
@@ -716,7 +687,7 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
     DeviceInfo* info;
     int8mm_status st = current_device(&dev, &info);
     if (st != INT8MM_OK) return st;
-    if (use_decode && !decode_plan(M, K, N, info, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (use_decode && !decode_plan(M, K, N, max_outliers, info->sm_count, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* b = static_cast<uint8_t*>(ws);
@@ -775,11 +746,14 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
         e = launch(k_detect, dim3(gx, gy), dim3(256), 0, s, false, X, M, K, threshold, rows, mask);
     }
     if (e == cudaSuccess) {
-        if (K <= 256 * 8 * kQRChunks) {
-            // one row per block, held in registers: X read once
+        const int kc = cdiv(K / 8, 256);  // 8-column chunks per thread
+        if (kc <= 8) {
+            // one row per block, held in registers (X read once)
             const size_t smem = (size_t)cdiv(K, 32) * 2 * 4;
-            e = launch(k_quant_rows_reg, dim3(M), dim3(256), smem, s, true, X, M, K, (const uint32_t*)mask,
-                       max_outliers, kp, xq, ra, xo, idx, n_out, status);
+            auto kern = kc <= 2 ? k_quant_rows_reg<2> : kc <= 4 ? k_quant_rows_reg<4>
+                      : kc <= 6 ? k_quant_rows_reg<6> : k_quant_rows_reg<8>;
+            e = launch(kern, dim3(M), dim3(256), smem, s, true, X, M, K, (const uint32_t*)mask, max_outliers, kp,
+                       xq, ra, xo, idx, n_out, status);
         } else {
             // mask words, their prefix counts, and one flag word per 2048-column window
             const size_t smem = ((size_t)cdiv(K, 32) * 2 + (size_t)cdiv(K, 2048)) * 4;
@@ -868,13 +842,13 @@ int8mm_status int8mm_forward_decode_noalloc(const uint16_t* X, int M, const int8
     const NoAllocLayout L = noalloc_layout(M, K);
     if (L.total > kNoAllocBytes) return INT8MM_ERR_INVALID_ARGUMENT;
     DecodePlan dp{};
-    if (!decode_plan(M, K, N, nullptr, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!decode_plan(M, K, N, cap, 1 << 20, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
 
     int dev;
     DeviceInfo* info;
     int8mm_status st = current_device(&dev, &info);
     if (st != INT8MM_OK) return st;
-    if (!decode_plan(M, K, N, info, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
+    if (!decode_plan(M, K, N, cap, info->sm_count, &dp)) return INT8MM_ERR_INVALID_ARGUMENT;
     uint8_t* b = nullptr;
     st = noalloc_scratch(dev, &b);
     if (st != INT8MM_OK) return st;
@@ -937,10 +911,17 @@ int8mm_status int8mm_block_dequantize(const int8_t* q, const float* absmax, int6
     DeviceInfo* info;
     int8mm_status st = current_device(&dev, &info);
     if (st != INT8MM_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (B >= 256) {
+        // a table of the block's 129 values per block, then look-ups
+        const long long nblocks = (n + B - 1) / B;
+        const int grid = (int)std::max<long long>(1, std::min<long long>(nblocks, (long long)info->sm_count * 8));
+        return cuda_status(launch(k_block_dequant_table, dim3(grid), dim3(256), 0, s, false, q, absmax, (long long)n, B,
+                                  out));
+    }
     const long long nq = (n + 3) / 4;
     const int grid = (int)std::max<long long>(1, std::min<long long>((nq + 255) / 256, (long long)info->sm_count * 16));
-    return cuda_status(launch(k_block_dequant, dim3(grid), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream), false,
-                              q, absmax, (long long)n, B, out));
+    return cuda_status(launch(k_block_dequant, dim3(grid), dim3(256), 0, s, false, q, absmax, (long long)n, B, out));
 }
 
 size_t int8mm_int4_weight_bytes(int K, int N, int G) {

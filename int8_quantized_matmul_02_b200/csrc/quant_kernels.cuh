@@ -427,13 +427,15 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
 }
 
 // k_quant_rows with one row per 256-thread block, the row held in registers
-// (up to kQRChunks 8-column chunks per thread: K <= 256 * 8 * kQRChunks), so X
-// is read from memory once: the loads are issued first and land while the
-// block takes the prefix counts of the outlier bitmask; the row maximum is one
-// block reduction, and the codes go out in the same pass (each warp stores
-// 256 contiguous bytes per step).  Same results as k_quant_rows.
-constexpr int kQRChunks = 8;
-
+// (kC 8-column chunks per thread, K <= 2048 * kC), so X is read from memory
+// once.  The row's loads go out first; the block copies the outlier bitmask to
+// shared memory (barrier 1); warp 0 then forms the words' prefix counts while
+// every warp takes its part of the row maximum over the non-outlier columns,
+// and one more barrier (2) publishes both; the codes and the outlier values
+// follow in the same pass (each warp stores 256 contiguous bytes per step).
+// Block 0 also writes the outlier list, the count and the overflow flag.  Same
+// results as k_quant_rows.
+template <int kC>
 __global__ void __launch_bounds__(256) k_quant_rows_reg(const uint16_t* __restrict__ X, int M, int K,
                                                         const uint32_t* __restrict__ mask, int cap, int kp,
                                                         int8_t* __restrict__ Xq, float* __restrict__ ra,
@@ -443,8 +445,8 @@ __global__ void __launch_bounds__(256) k_quant_rows_reg(const uint16_t* __restri
     const int nw = (K + 31) / 32;
     uint32_t* smask = qsm;
     int* spre = reinterpret_cast<int*>(qsm + nw);
-    __shared__ int red[8];
     __shared__ uint32_t bmax[8];
+    __shared__ int total_sh;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int m = blockIdx.x;
     const int nchunk = K / 8;
@@ -452,20 +454,36 @@ __global__ void __launch_bounds__(256) k_quant_rows_reg(const uint16_t* __restri
     pdl_wait();  // the outlier bitmask comes from k_detect
     pdl_launch_dependents();
     const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)m * K);
-    uint4 v[kQRChunks];
+    uint4 v[kC];
 #pragma unroll
-    for (int i = 0; i < kQRChunks; ++i) {
+    for (int i = 0; i < kC; ++i) {
         const int c = tid + 256 * i;
         if (c < nchunk) v[i] = __ldg(xr + c);
     }
-    const int total = load_mask_prefix(mask, nw, smask, spre, red);
-    const int n_eff = min(total, cap);
-    const int n_pad = min(kp, (n_eff + 63) / 64 * 64);
-    if (m == 0) write_outlier_list(smask, spre, nw, total, cap, idx, n_out, status);
-
+    for (int w = tid; w < nw; w += 256) smask[w] = __ldg(mask + w);
+    __syncthreads();  // (1) the bitmask
+    if (warp == 0) {
+        // exclusive prefix counts of the words, lane l taking words [l*per, (l+1)*per)
+        const int per = (nw + 31) / 32;
+        const int w0 = min(nw, lane * per), w1 = min(nw, w0 + per);
+        int cnt = 0;
+        for (int w = w0; w < w1; ++w) cnt += __popc(smask[w]);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        int run = incl - cnt;
+        for (int w = w0; w < w1; ++w) {
+            spre[w] = run;
+            run += __popc(smask[w]);
+        }
+        if (lane == 31) total_sh = incl;
+    }
     uint32_t amax = 0;
 #pragma unroll
-    for (int i = 0; i < kQRChunks; ++i) {
+    for (int i = 0; i < kC; ++i) {
         const int c = tid + 256 * i;
         if (c < nchunk) {
             const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
@@ -474,7 +492,11 @@ __global__ void __launch_bounds__(256) k_quant_rows_reg(const uint16_t* __restri
     }
     amax = __reduce_max_sync(0xffffffffu, amax);
     if (lane == 0) bmax[warp] = amax;
-    __syncthreads();
+    __syncthreads();  // (2) the prefix counts, the total and the warps' maxima
+    const int total = total_sh;
+    const int n_eff = min(total, cap);
+    const int n_pad = min(kp, (n_eff + 63) / 64 * 64);
+    if (m == 0) write_outlier_list(smask, spre, nw, total, cap, idx, n_out, status);
     amax = 0;
 #pragma unroll
     for (int w = 0; w < 8; ++w) amax = max(amax, bmax[w]);
@@ -484,7 +506,7 @@ __global__ void __launch_bounds__(256) k_quant_rows_reg(const uint16_t* __restri
     uint2* qr = reinterpret_cast<uint2*>(Xq + (size_t)m * K);
     uint16_t* xo_row = Xo + (size_t)m * kp;
 #pragma unroll
-    for (int i = 0; i < kQRChunks; ++i) {
+    for (int i = 0; i < kC; ++i) {
         const int c = tid + 256 * i;
         if (c < nchunk) {
             const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
