@@ -84,42 +84,75 @@ def dist_info():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons sampled during the timed region.
+
+    The sampler polls every 20 ms from a reader thread that stamps each line
+    with the host clock. Entering waits until the first sample has arrived, so
+    polling is live when timing starts; `mark()` brackets the timed region and
+    `summary()` keeps the samples inside it (the two nearest ones when the
+    region is shorter than two polling periods, and says so)."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_MS = 20
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.samples = []          # (host time, line)
+        self.region = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            if line.strip():
+                self.samples.append((time.perf_counter(), line))
 
     def __enter__(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", str(self.PERIOD_MS)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return self
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        t_end = time.perf_counter() + 3.0
+        while not self.samples and time.perf_counter() < t_end and self.proc.poll() is None:
+            time.sleep(0.005)
+        self.t_enter = time.perf_counter()
         return self
 
+    def mark(self, which: str):
+        """Host time of the start ('start') or end ('end') of the timed region."""
+        now = time.perf_counter()
+        if which == "start":
+            self.region = [now, None]
+        else:
+            self.region[1] = now
+
     def __exit__(self, *exc):
-        self.lines = []
+        if self.region is None:
+            self.region = [self.t_enter if self.proc else 0.0, time.perf_counter()]
+        elif self.region[1] is None:
+            self.region[1] = time.perf_counter()
         if self.proc is not None:
-            time.sleep(0.25)
+            time.sleep(2.5 * self.PERIOD_MS / 1000.0)
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+                self.proc.wait()
+            self.thread.join(timeout=5)
         return False
 
     def summary(self):
-        sms, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        parsed = []
+        for t, line in list(self.samples):
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 8:
                 continue
@@ -127,16 +160,21 @@ class ClockSampler:
                 sm, smax = float(parts[0]), float(parts[1])
             except ValueError:
                 continue
-            sms.append(sm)
-            mx = smax
-            for n, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sms:
+            parsed.append((t, sm, smax, [n for n, v in zip(names, parts[4:8]) if v.lower() == "active"]))
+        if not parsed or self.region is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        loaded = [s for s in sms if s > 0.5 * max(sms)] or sms
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sms)}
+        t0, t1 = self.region
+        inside = [p for p in parsed if t0 <= p[0] <= t1]
+        basis = "inside the timed region"
+        if len(inside) < 2:
+            mid = 0.5 * (t0 + t1)
+            inside = sorted(parsed, key=lambda p: abs(p[0] - mid))[:2]
+            basis = "the two samples nearest the timed region (shorter than two polling periods)"
+        sms = [p[1] for p in inside]
+        reasons = sorted({r for p in inside for r in p[3]})
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": inside[-1][2], "reasons": reasons,
+                "samples": len(inside), "period_ms": self.PERIOD_MS, "region_ms": round(1000 * (t1 - t0), 1),
+                "basis": basis}
 
 
 KERNEL_SOURCES = {
@@ -258,11 +296,13 @@ def run_gemm_workload(wl, steps: int, warmup: int, dev, rank: int, cap: int):
     barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        clk.mark("start")
         t0.record(stream)
         for i in range(steps):
             step(evs[i])
         t1.record(stream)
         torch.cuda.synchronize(dev)
+        clk.mark("end")
     barrier()
     total_ms = t0.elapsed_time(t1)
     kern_ms = [a.elapsed_time(b) for a, b in evs]
@@ -480,11 +520,13 @@ def run_grouped(wl, G: int, steps: int, warmup: int, dev, cap: int):
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        clk.mark("start")
         a.record(stream)
         for i in range(steps):
             step(evs[i])
         b.record(stream)
         torch.cuda.synchronize(dev)
+        clk.mark("end")
     st, n_o = i8.device_status(ws)
     if st != 0:
         raise RuntimeError(f"grouped device status {st}")
@@ -563,7 +605,7 @@ def main():
     global _pg
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="175b", choices=sorted(synth.WORKLOADS))

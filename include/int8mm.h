@@ -36,8 +36,9 @@
  *   - "device" pointers point to memory of the current CUDA device; the
  *     caller allocates and owns all memory.  The library calls no device
  *     allocator.  Between calls it keeps only a per-device cache of device
- *     properties on the host and, for int8mm_forward_decode_noalloc alone,
- *     the static scratch array described with that function.
+ *     properties on the host, the copy stream and events of
+ *     int8mm_forward_host and, for int8mm_forward_decode_noalloc alone, the
+ *     static scratch array described with that function.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Calls are stream-ordered and do not synchronise the host,
  *     except where a function says so.
@@ -161,6 +162,27 @@ enum { INT8MM_TEST_WITHHOLD_SIGNAL = 1 };
 int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w, float threshold,
                                 int max_outliers, uint16_t* Y, void* ws, size_t ws_bytes,
                                 const int8mm_forward_opts* opts, void* stream);
+
+/* int8mm_forward from and to host memory (same method, LLM.int8() abstract).
+ *   x_host  HOST, M x K fp16, read by a host-to-device copy into x_dev;
+ *   y_host  HOST, M x N fp16, written by device-to-host copies from y_dev;
+ *   x_dev   DEVICE, M x K fp16 staging buffer (16-byte aligned), caller-owned;
+ *   y_dev   DEVICE, M x N fp16 staging buffer (16-byte aligned), caller-owned;
+ *   other arguments as for int8mm_forward.
+ * Page-locked (pinned) host buffers let the copies run asynchronously; with
+ * pageable ones the driver stages them and the call may block the host.
+ * On the tiled path (M > 16) the product is computed in bands of whole
+ * 256-row tiles (at most 8 bands) and each band's rows are copied back on a
+ * second stream, owned by the library (one per device, created at the first
+ * call on that device together with its events), while the next band is
+ * computed; the decode path copies Y back after its one kernel.  All the
+ * call's work is ordered on `stream`: once the stream has reached the end of
+ * the call (e.g. cudaStreamSynchronize returns), y_host holds Y.  The host
+ * buffers must not be changed or freed before that.  Device-side errors are
+ * read with int8mm_get_device_status, as for int8mm_forward. */
+int8mm_status int8mm_forward_host(const uint16_t* x_host, int M, const int8mm_weight* w, float threshold,
+                                  int max_outliers, uint16_t* y_host, uint16_t* x_dev, uint16_t* y_dev,
+                                  void* ws, size_t ws_bytes, void* stream);
 
 /* Device pointers to the intermediates a forward leaves in its workspace. */
 typedef struct {
@@ -289,6 +311,9 @@ int8mm_status int8mm_prepare_weight_int4(const uint16_t* W, int K, int N, int G,
 /* Y (device, M x N fp16) = X (device, M x K fp16) times the 4-bit weight,
  * 1 <= M <= 16:  y[m,n] = sum_k x[m,k] * (q[n,k] * absmax[n,g(k)] / 7), the
  * products on the tensor cores with fp32 sums, rounded to fp16 once.
+ * The kernel keeps its share of X in shared memory, which bounds K: K <=
+ * 40960 for M <= 8 and K <= 12288 for 9 <= M <= 16; longer K returns
+ * INT8MM_ERR_INVALID_ARGUMENT.
  * status: device int32 word, zero before the call; a wait in the kernel that
  * runs out sets bit 0 (INT8MM_ERR_TIMEOUT: outputs invalid).  Stream-ordered
  * (programmatic dependent launch: the weight stream of a call starts while

@@ -148,22 +148,46 @@ def forward(X: torch.Tensor, w: PreparedWeight, threshold: float = 6.0, *, max_o
             out: torch.Tensor | None = None, workspace: Workspace | None = None, path: str = "auto",
             acc_out: torch.Tensor | None = None, wait_limit_ns: int = 0, test_flags: int = 0,
             stream=None) -> torch.Tensor:
-    """Y = X W by LLM.int8().  X: M x K fp16.  A CPU X is copied to the GPU and
-    the result copied back (end to end); a CUDA X stays on its device."""
+    """Y = X W by LLM.int8().  X: M x K fp16.  A CPU X goes through
+    int8mm_forward_host (copy in, product, copy back in row bands that overlap
+    the product) and a CPU Y (``out``, pinned if given, else a new pinned
+    tensor) is returned once it is complete; a CUDA X stays on its device."""
     lib = _abi.load()
     on_host = not X.is_cuda
     dev = w.buf.device
     if X.dtype != torch.float16 or X.dim() != 2 or X.shape[1] != w.K:
         raise ValueError(f"X must be float16 of shape (M, {w.K})")
-    Xd = X.to(dev, non_blocking=True) if on_host else X
-    if not Xd.is_contiguous():
+    if not X.is_contiguous():
         raise ValueError("X must be contiguous")
-    M = Xd.shape[0]
+    M = X.shape[0]
+    if on_host:
+        if acc_out is not None or path != "auto" or wait_limit_ns or test_flags:
+            raise ValueError("a host X takes the default path and options")
+        if workspace is None:
+            workspace = Workspace(M, w.K, w.N, max_outliers, device=dev)
+        if (workspace.M, workspace.K, workspace.N) != (M, w.K, w.N):
+            raise ValueError("workspace was made for another shape")
+        host = out if out is not None else torch.empty(M, w.N, dtype=torch.float16, pin_memory=True)
+        if host.is_cuda or host.shape != (M, w.N) or host.dtype != torch.float16 or not host.is_contiguous():
+            raise ValueError("out must be a contiguous CPU float16 tensor of shape (M, N) for a host X")
+        Xd = torch.empty(M, w.K, dtype=torch.float16, device=dev)
+        Yd = torch.empty(M, w.N, dtype=torch.float16, device=dev)
+        with torch.cuda.device(dev):
+            st = stream or torch.cuda.current_stream()
+            _abi.check(lib.int8mm_forward_host(ctypes.c_void_p(X.data_ptr()), M, ctypes.byref(w.struct),
+                                               float(threshold), workspace.max_outliers,
+                                               ctypes.c_void_p(host.data_ptr()), ctypes.c_void_p(Xd.data_ptr()),
+                                               ctypes.c_void_p(Yd.data_ptr()),
+                                               ctypes.c_void_p(workspace.buf.data_ptr()), workspace.nbytes,
+                                               _stream(stream)), "int8mm_forward_host")
+            st.synchronize()
+        return host
+    Xd = X
     if workspace is None:
         workspace = Workspace(M, w.K, w.N, max_outliers, device=dev)
     if (workspace.M, workspace.K, workspace.N) != (M, w.K, w.N):
         raise ValueError("workspace was made for another shape")
-    Y = out if (out is not None and not on_host) else torch.empty(M, w.N, dtype=torch.float16, device=dev)
+    Y = out if out is not None else torch.empty(M, w.N, dtype=torch.float16, device=dev)
     opts = _abi.ForwardOpts(_PATHS[path], ctypes.c_void_p(acc_out.data_ptr()) if acc_out is not None else None,
                             int(wait_limit_ns), None, None, int(test_flags))
     with torch.cuda.device(dev):
@@ -171,11 +195,6 @@ def forward(X: torch.Tensor, w: PreparedWeight, threshold: float = 6.0, *, max_o
                                          workspace.max_outliers, ctypes.c_void_p(Y.data_ptr()),
                                          ctypes.c_void_p(workspace.buf.data_ptr()), workspace.nbytes,
                                          ctypes.byref(opts), _stream(stream)), "int8mm_forward")
-    if on_host:
-        host = out if out is not None else torch.empty(M, w.N, dtype=torch.float16, pin_memory=True)
-        host.copy_(Y, non_blocking=True)
-        (stream or torch.cuda.current_stream()).synchronize()
-        return host
     return Y
 
 

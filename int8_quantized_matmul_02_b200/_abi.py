@@ -28,6 +28,7 @@ PATH_AUTO, PATH_GEMM, PATH_DECODE, PATH_GEMM_1SM = 0, 1, 2, 3
 EXPORTS = (
     "int8mm_status_string", "int8mm_version", "int8mm_weight_bytes", "int8mm_prepare_weight",
     "int8mm_workspace_bytes", "int8mm_workspace_init", "int8mm_forward", "int8mm_forward_ex",
+    "int8mm_forward_host",
     "int8mm_workspace_view_get", "int8mm_get_device_status",
     "int8mm_forward_decode_noalloc", "int8mm_noalloc_device_status",
     "int8mm_block_quantize", "int8mm_block_dequantize",
@@ -110,6 +111,8 @@ def load(path: str | None = None):
     lib.int8mm_forward.restype = I
     lib.int8mm_forward_ex.argtypes = [P, I, ctypes.POINTER(Weight), F, I, P, P, S, ctypes.POINTER(ForwardOpts), P]
     lib.int8mm_forward_ex.restype = I
+    lib.int8mm_forward_host.argtypes = [P, I, ctypes.POINTER(Weight), F, I, P, P, P, P, S, P]
+    lib.int8mm_forward_host.restype = I
     lib.int8mm_workspace_view_get.argtypes = [P, S, I, I, I, I, ctypes.POINTER(WorkspaceView)]
     lib.int8mm_workspace_view_get.restype = I
     lib.int8mm_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]

@@ -15,7 +15,9 @@
 // The accumulation of a group ends in one of two s32 TMEM accumulators; while
 // the tensor cores fill the other with the next group, the epilogue drains
 // it, applies the group's constants (acc * (ra / 127^2) * ca, one multiply and
-// one fused multiply-add per element) and adds the result to the tile's
+// one fused multiply-add per element, in packed pairs; for G <= 256 the
+// int32 sums become floats by an exact add-and-subtract instead of the
+// conversion unit, whose rate is a fraction of the FMA rate) and adds the result to the tile's
 // running fp32 sums, which each epilogue thread keeps in registers (its row,
 // 64 columns).  With outlier columns the sums go to TMEM (columns 256-383)
 // once per tile, and the fp16 outlier product accumulates onto them there.
@@ -58,6 +60,41 @@ constexpr int kGGCaBytes = 2 * 64 * 4;            // per epilogue warp: two grou
 constexpr int kGGSmemBytes =
     1024 + kGGStages * kGGStageBytes + kGGEpiWarps * (2 * kGemmEpiBufBytes + kGGCaBytes) + 256;
 constexpr uint32_t kGGSumCol = 256;                // running fp32 sums; accumulators at 0 and 128
+
+// Pairs of fp32 lanes in one instruction (sm_100 packed f32x2 arithmetic;
+// each lane rounds as its scalar counterpart does).
+__device__ __forceinline__ void mul2_rn(float& d0, float& d1, float a0, float a1, float b) {
+    asm("{\n\t.reg .b64 x, y;\n\t"
+        "mov.b64 x, {%2, %3};\n\t"
+        "mov.b64 y, {%4, %4};\n\t"
+        "mul.rn.f32x2 x, x, y;\n\t"
+        "mov.b64 {%0, %1}, x;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b));
+}
+__device__ __forceinline__ void fma2_rn(float& acc0, float& acc1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 x, y, z;\n\t"
+        "mov.b64 x, {%2, %3};\n\t"
+        "mov.b64 y, {%4, %5};\n\t"
+        "mov.b64 z, {%0, %1};\n\t"
+        "fma.rn.f32x2 z, x, y, z;\n\t"
+        "mov.b64 {%0, %1}, z;\n\t}"
+        : "+f"(acc0), "+f"(acc1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// float(a) for |a| < 2^22 without the conversion unit: a + 1.5 * 2^23 read as
+// a float lies in [2^23, 2^24), where the spacing is 1, so it is exactly
+// 1.5 * 2^23 + a, and the subtraction of 1.5 * 2^23 is exact too.
+__device__ __forceinline__ void small_int_to_float2(float& f0, float& f1, uint32_t a0, uint32_t a1) {
+    const float b0 = __uint_as_float(a0 + 0x4B400000u), b1 = __uint_as_float(a1 + 0x4B400000u);
+    asm("{\n\t.reg .b64 x, y;\n\t"
+        "mov.b64 x, {%2, %3};\n\t"
+        "mov.b64 y, {%4, %4};\n\t"
+        "add.rn.f32x2 x, x, y;\n\t"
+        "mov.b64 {%0, %1}, x;\n\t}"
+        : "=f"(f0), "=f"(f1)
+        : "f"(b0), "f"(b1), "f"(-12582912.0f));
+}
 
 template <bool kWriteAcc>
 __global__ void __launch_bounds__(kGGThreads, 1)
@@ -276,6 +313,7 @@ __global__ void __launch_bounds__(kGGThreads, 1)
                 asm volatile("cp.async.commit_group;" ::: "memory");
             };
             fetch_ca(0);
+            const bool small_group = gp.G <= 256;
             float ra_next = row < p.M ? gp.ra[(size_t)row * ng] : 0.0f;
             for (int g = 0; g < ng; ++g) {
                 if (!__all_sync(0xffffffffu, wait_bounded_cluster(&tfull[acc], acc_phase, wctx))) {
@@ -286,22 +324,24 @@ __global__ void __launch_bounds__(kGGThreads, 1)
                 const uint32_t tacc = tmem_base + lane_off + (uint32_t)(acc * kGGBN + half * 64);
                 // ra / 127^2 once per row and group; each term is acc * (ra / 127^2) * ca
                 const float rs = __fmul_rn(ra_next, 1.0f / 16129.0f);
-                if (g + 1 < ng) {
-                    fetch_ca(g + 1);
-                    ra_next = row < p.M ? gp.ra[(size_t)row * ng + g + 1] : 0.0f;
-                } else {
-                    asm volatile("cp.async.commit_group;" ::: "memory");  // keeps the group count in step
-                }
                 uint32_t r[64];
                 tmem_ld32(tacc, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
                 tmem_ld32(tacc + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(tempty_even[acc]);  // the accumulator is free
+                // the accumulator is free; the release is issued before the next
+                // group's constant loads so that it does not wait for them
+                if (lane == 0) mbar_arrive_cluster(tempty_even[acc]);
                 if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1;
+                }
+                if (g + 1 < ng) {
+                    fetch_ca(g + 1);
+                    ra_next = row < p.M ? gp.ra[(size_t)row * ng + g + 1] : 0.0f;
+                } else {
+                    asm volatile("cp.async.commit_group;" ::: "memory");  // keeps the group count in step
                 }
                 if (kWriteAcc && row < p.M) {
 #pragma unroll 4
@@ -311,13 +351,31 @@ __global__ void __launch_bounds__(kGGThreads, 1)
                 asm volatile("cp.async.wait_group 1;" ::: "memory");  // this group's constants have landed
                 __syncwarp();
                 const float4* cs = reinterpret_cast<const float4*>(wca + (g & 1) * 64);
+                // v += RN(float(acc) * rs) * ca, two columns per instruction;
+                // float(acc) is exact either way: a group sum is at most
+                // 127^2 G in magnitude, below 2^22 for G <= 256
+                if (small_group) {
 #pragma unroll
-                for (int q4 = 0; q4 < 16; ++q4) {
-                    const float4 c4 = cs[q4];
-                    v[4 * q4 + 0] = fmaf(__fmul_rn((float)(int32_t)r[4 * q4 + 0], rs), c4.x, v[4 * q4 + 0]);
-                    v[4 * q4 + 1] = fmaf(__fmul_rn((float)(int32_t)r[4 * q4 + 1], rs), c4.y, v[4 * q4 + 1]);
-                    v[4 * q4 + 2] = fmaf(__fmul_rn((float)(int32_t)r[4 * q4 + 2], rs), c4.z, v[4 * q4 + 2]);
-                    v[4 * q4 + 3] = fmaf(__fmul_rn((float)(int32_t)r[4 * q4 + 3], rs), c4.w, v[4 * q4 + 3]);
+                    for (int q4 = 0; q4 < 16; ++q4) {
+                        const float4 c4 = cs[q4];
+                        float f0, f1, f2, f3;
+                        small_int_to_float2(f0, f1, r[4 * q4 + 0], r[4 * q4 + 1]);
+                        small_int_to_float2(f2, f3, r[4 * q4 + 2], r[4 * q4 + 3]);
+                        mul2_rn(f0, f1, f0, f1, rs);
+                        mul2_rn(f2, f3, f2, f3, rs);
+                        fma2_rn(v[4 * q4 + 0], v[4 * q4 + 1], f0, f1, c4.x, c4.y);
+                        fma2_rn(v[4 * q4 + 2], v[4 * q4 + 3], f2, f3, c4.z, c4.w);
+                    }
+                } else {
+#pragma unroll
+                    for (int q4 = 0; q4 < 16; ++q4) {
+                        const float4 c4 = cs[q4];
+                        float f0, f1, f2, f3;
+                        mul2_rn(f0, f1, (float)(int32_t)r[4 * q4 + 0], (float)(int32_t)r[4 * q4 + 1], rs);
+                        mul2_rn(f2, f3, (float)(int32_t)r[4 * q4 + 2], (float)(int32_t)r[4 * q4 + 3], rs);
+                        fma2_rn(v[4 * q4 + 0], v[4 * q4 + 1], f0, f1, c4.x, c4.y);
+                        fma2_rn(v[4 * q4 + 2], v[4 * q4 + 3], f2, f3, c4.z, c4.w);
+                    }
                 }
                 __syncwarp();  // every lane has read the slot before it is refilled
             }

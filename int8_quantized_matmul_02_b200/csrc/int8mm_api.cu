@@ -203,20 +203,42 @@ WeightLayout grouped_weight_layout(int K, int N, int G, int n_keep) {
 }
 
 struct WsLayout {
-    size_t status, n_out, mask, idx, ra, xq, xo, wo, total;
+    size_t status, n_out, ticket, part, mask, spre, idx, ra, xq, xo, wo, total;
     int kp;
 };
+
+// Grid of k_detect: gx blocks of 256 columns by gy row splits of `rows` rows
+// (a multiple of 8), about kDetectBlocks blocks in all; a fixed budget (not
+// the device's SM count) so that the workspace size depends on the shape only.
+constexpr int kDetectBlocks = 592;
+struct DetectGrid {
+    int gx, gy, rows;
+};
+DetectGrid detect_grid(int M, int K) {
+    DetectGrid d;
+    d.gx = cdiv(K, 256);
+    d.gy = std::max(1, std::min(cdiv(M, 8), cdiv(kDetectBlocks, d.gx)));
+    d.rows = (cdiv(M, d.gy) + 7) / 8 * 8;
+    d.gy = cdiv(M, d.rows);
+    return d;
+}
 
 // ng: constants per row of X (1 vector-wise, K / G group-wise)
 WsLayout ws_layout(int M, int K, int N, int max_outliers, int ng = 1) {
     WsLayout L{};
     L.kp = (max_outliers + 63) / 64 * 64;
+    const size_t nw = (size_t)cdiv(K, 32);
     size_t o = 0;
     L.status = 0;
     L.n_out = 4;
+    L.ticket = 8;
     o = 256;
+    L.part = o;
+    o = align_up(o + (size_t)detect_grid(M, K).gy * nw * 4, 256);
     L.mask = o;
-    o = align_up(o + (size_t)cdiv(K, 32) * 4, 256);
+    o = align_up(o + nw * 4, 256);
+    L.spre = o;
+    o = align_up(o + nw * 4, 256);
     L.idx = o;
     o = align_up(o + (size_t)K * 4, 256);
     L.ra = o;
@@ -230,6 +252,10 @@ WsLayout ws_layout(int M, int K, int N, int max_outliers, int ng = 1) {
     L.total = o;
     return L;
 }
+
+// Outlier detection of the tiled paths (k_detect, finalised by its last block).
+cudaError_t launch_detect(const uint16_t* X, int M, int K, float threshold, const WsLayout& L, uint8_t* b, int cap,
+                          cudaStream_t s);
 
 bool shape_ok(int M, int K, int N) {
     return M >= 1 && K >= 16 && N >= 16 && K % 16 == 0 && N % 16 == 0 && K <= kMaxK;
@@ -267,6 +293,18 @@ cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_
 template <typename Kern, typename... Args>
 cudaError_t launch(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl, Args... args) {
     return launch_ex(kern, grid, block, smem, st, pdl, 0, args...);
+}
+
+// Launched without PDL: its per-split words and ticket are reused from the
+// previous call, whose kernels must have finished.
+cudaError_t launch_detect(const uint16_t* X, int M, int K, float threshold, const WsLayout& L, uint8_t* b, int cap,
+                          cudaStream_t s) {
+    const DetectGrid d = detect_grid(M, K);
+    return launch(k_detect, dim3(d.gx, d.gy), dim3(256), 0, s, false, X, M, K, threshold, d.rows,
+                  reinterpret_cast<uint32_t*>(b + L.part), reinterpret_cast<uint32_t*>(b + L.mask),
+                  reinterpret_cast<int32_t*>(b + L.spre), reinterpret_cast<int32_t*>(b + L.idx),
+                  reinterpret_cast<int32_t*>(b + L.n_out), cap, reinterpret_cast<int*>(b + L.status),
+                  reinterpret_cast<unsigned*>(b + L.ticket));
 }
 
 int8mm_status cuda_status(cudaError_t e) {
@@ -437,36 +475,44 @@ bool int4_shape_ok(int K, int N, int G) {
 
 // Plan of the 4-bit kernel: clusters of `cluster` CTAs split K in 256-k
 // boxes, tiles shared out evenly (at most `cluster` per cluster), one CTA per
-// SM (the kernel takes the whole TMEM), one wave when the tiles allow.
+// SM (its shared memory), one wave when the tiles allow.
 struct Int4Plan {
-    int cluster, clusters, stages, xrows, grid;
-    uint32_t tmem_cols, off_x, off_red, off_bars, bytes;
+    int cluster, clusters, stages, xrows, grid, aslots;
+    uint32_t tmem_cols, off_a, off_x, off_red, off_bars, bytes;
 };
 
+// The first fit in this order: clusters of 4, then 8 CTAs (more CTAs share
+// the K range, so less of X per CTA); three A operands, then two; the most
+// ring stages up to 12 (at least 3).  The kernel keeps its K range of X in
+// shared memory, so K is bounded: with 8-row X boxes (M <= 8) up to about
+// 40 K, with 16-row boxes (M <= 16) up to about 12 K.
 bool int4_plan(int M, int K, int N, DeviceInfo* dev, Int4Plan* P) {
     if (M < 1 || M > kInt4MaxRows) return false;
     const int kbt = cdiv(K, kI4BoxK);
     const int tiles = cdiv(N, kI4TileN);
     const int xrows = M <= 8 ? 8 : 16;
-    // one CTA per SM (the kernel takes the whole TMEM)
-    for (size_t cap : {(size_t)kMaxSmemOptin}) {
-        for (int c : {4, 8}) {
-            const int cl = std::min(c, kbt);
-            int ncl = std::max(1, std::min(tiles, cluster_capacity(dev, cl)));
-            if (cdiv(tiles, ncl) > cl) ncl = cdiv(tiles, cl);
-            const size_t xb = (size_t)cdiv(kbt, cl) * (kI4BoxK / 64) * xrows * 128 + 1024;  // + the row-8 overhang
-            const size_t red = (size_t)cl * kI4TileN * xrows * 4;  // a slot per peer and one for its own sums
+    const size_t cap = (size_t)kMaxSmemOptin;
+    for (int c : {4, 8}) {
+        const int cl = std::min(c, kbt);
+        int ncl = std::max(1, std::min(tiles, cluster_capacity(dev, cl)));
+        if (cdiv(tiles, ncl) > cl) ncl = cdiv(tiles, cl);
+        const size_t xb = (size_t)cdiv(kbt, cl) * (kI4BoxK / 64) * xrows * 128 + 1024;  // + the row-8 overhang
+        const size_t red = (size_t)cl * kI4TileN * xrows * 4;  // a slot per peer and one for its own sums
+        for (int as = kI4ASlots; as >= 2; --as) {
             for (int s = 12; s >= 3; --s) {
                 const size_t bars = (size_t)(2 * s + 2 * kI4ASlots + 2 * kI4DSlots + 3) * 8 + 64;
-                const size_t total = 1024 + (size_t)s * kI4StageBytes + xb + red + bars;
+                const size_t total = 1024 + (size_t)s * kI4StageBytes + (size_t)as * kI4ABytes + xb + red + bars;
                 if (total > cap) continue;
                 P->cluster = cl;
                 P->clusters = ncl;
                 P->stages = s;
                 P->xrows = xrows;
                 P->grid = cl * ncl;
+                P->aslots = as;
                 P->tmem_cols = kI4TmemCols;
                 size_t o = (size_t)s * kI4StageBytes;
+                P->off_a = (uint32_t)o;
+                o += (size_t)as * kI4ABytes;
                 P->off_x = (uint32_t)o;
                 o += xb;
                 P->off_red = (uint32_t)o;
@@ -649,13 +695,53 @@ int8mm_status int8mm_get_device_status(const void* ws, void* stream, int32_t* n_
     return INT8MM_OK;
 }
 
-int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w, float threshold,
-                                int max_outliers, uint16_t* Y, void* ws, size_t ws_bytes,
-                                const int8mm_forward_opts* opts, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Per-device copy stream and events of int8mm_forward_host.
+constexpr int kHostBands = 8;
+struct HostPipe {
+    bool ready = false;
+    cudaStream_t copy = nullptr;
+    cudaEvent_t band_done[kHostBands] = {};
+    cudaEvent_t copies_done = nullptr;
+};
+std::mutex g_host_mu;
+HostPipe g_host_pipe[64];
+
+// Copy-back of Y to host memory in row bands (int8mm_forward_host): the tiled
+// path runs its GEMM one band at a time and queues each band's copy on a
+// second stream as soon as that band is written.
+struct HostCopy {
+    uint16_t* y_host;
+    cudaStream_t copy;
+    cudaEvent_t* band_done;  // one per band, recorded on the compute stream
+    cudaEvent_t copies_done; // recorded on the copy stream after the last band
+    int bands;
+};
+
+// The argument checks of a forward that need no options.
+int8mm_status forward_check(const uint16_t* X, int M, const int8mm_weight* w, float threshold, int max_outliers,
+                            const uint16_t* Y, const void* ws, size_t ws_bytes) {
     if (!X || !w || !Y || !ws || !w->wq || !w->col_absmax || !w->keep_slot) return INT8MM_ERR_INVALID_ARGUMENT;
     const int K = w->K, N = w->N;
     if (!shape_ok(M, K, N) || max_outliers < 0 || max_outliers > K) return INT8MM_ERR_INVALID_ARGUMENT;
     if (!(threshold > 0.0f)) return INT8MM_ERR_INVALID_ARGUMENT;  // also rejects NaN
+    if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ws, 256) || !aligned(w->wq, 256))
+        return INT8MM_ERR_MISALIGNED;
+    if (ws_bytes < ws_layout(M, K, N, max_outliers).total) return INT8MM_ERR_WORKSPACE_TOO_SMALL;
+    return INT8MM_OK;
+}
+
+int8mm_status forward_core(const uint16_t* X, int M, const int8mm_weight* w, float threshold, int max_outliers,
+                           uint16_t* Y, void* ws, size_t ws_bytes, const int8mm_forward_opts* opts, void* stream,
+                           const HostCopy* hc) {
+    {
+        const int8mm_status chk = forward_check(X, M, w, threshold, max_outliers, Y, ws, ws_bytes);
+        if (chk != INT8MM_OK) return chk;
+    }
+    const int K = w->K, N = w->N;
     const int path = opts ? opts->path : INT8MM_PATH_AUTO;
     if (path < INT8MM_PATH_AUTO || path > INT8MM_PATH_GEMM_1SM) return INT8MM_ERR_INVALID_ARGUMENT;
     int32_t* acc_out = opts ? opts->acc_out : nullptr;
@@ -665,11 +751,8 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
     const bool timed = ev0 != nullptr;
     const uint32_t test_flags = opts ? opts->test_flags : 0u;
     const uint64_t wait_ns = (opts && opts->wait_limit_ns) ? opts->wait_limit_ns : kDefaultWaitNs;
-    if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ws, 256) || !aligned(w->wq, 256) ||
-        (acc_out && !aligned(acc_out, 16)))
-        return INT8MM_ERR_MISALIGNED;
+    if (acc_out && !aligned(acc_out, 16)) return INT8MM_ERR_MISALIGNED;
     const WsLayout L = ws_layout(M, K, N, max_outliers);
-    if (ws_bytes < L.total) return INT8MM_ERR_WORKSPACE_TOO_SMALL;
 
     // whether the decode kernel fits does not depend on the device; its grid does
     DecodePlan dp{};
@@ -716,63 +799,68 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
         cudaError_t e = timed ? cudaEventRecord(ev0, s) : cudaSuccess;
         if (e == cudaSuccess) e = launch_decode(dp, tm_w, p, s, !timed);
         if (e == cudaSuccess && timed) e = cudaEventRecord(ev1, s);
+        if (e == cudaSuccess && hc)
+            e = cudaMemcpyAsync(hc->y_host, Y, (size_t)M * N * 2, cudaMemcpyDeviceToHost, s);
         return cuda_status(e);
     }
 
     // ---- tiled path: detect -> quantise -> gather -> tcgen05 GEMM, PDL-chained
-    CUtensorMap tm_a, tm_b, tm_xo, tm_wo, tm_y;
+    CUtensorMap tm_b, tm_wo;
     const int kp = L.kp;
-    if (!make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, M, K, 128, kGemmBM) ||
-        !make_map(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq, K, N, K, 128, kGemmBN) ||
-        !make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Y, N, M, (uint64_t)N * 2, 64, 32))
-        return INT8MM_ERR_CUDA;
+    if (!make_map(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq, K, N, K, 128, kGemmBN)) return INT8MM_ERR_CUDA;
     if (kp > 0) {
-        if (!make_map(&tm_xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xo, kp, M, (uint64_t)kp * 2, 64, kGemmBM) ||
-            !make_map(&tm_wo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wo, kp, N, (uint64_t)kp * 2, 64, kGemmBN))
+        if (!make_map(&tm_wo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wo, kp, N, (uint64_t)kp * 2, 64, kGemmBN))
             return INT8MM_ERR_CUDA;
     } else {
-        tm_xo = tm_a;  // never dereferenced: no outlier slices without capacity
-        tm_wo = tm_b;
+        tm_wo = tm_b;  // never dereferenced: no outlier slices without capacity
     }
 
     const int sms = info->sm_count;
-    cudaError_t e;
-    {
-        const int gx = cdiv(K, 256);
-        int gy = std::max(1, std::min(cdiv(M, 8), cdiv(4 * sms, gx)));
-        int rows = cdiv(M, gy);
-        rows = (rows + 7) / 8 * 8;
-        gy = cdiv(M, rows);
-        e = launch(k_detect, dim3(gx, gy), dim3(256), 0, s, false, X, M, K, threshold, rows, mask);
-    }
+    cudaError_t e = launch_detect(X, M, K, threshold, L, b, max_outliers, s);
     if (e == cudaSuccess) {
         const int kc = cdiv(K / 8, 256);  // 8-column chunks per thread
         if (kc <= 8) {
-            // one row per block, held in registers (X read once)
-            const size_t smem = (size_t)cdiv(K, 32) * 2 * 4;
+            // one row per block, held in registers (X read once), with the
+            // outlier weight rows gathered by extra blocks in front of the rows
+            GatherArgs ga{(const int8_t*)w->wq, (const float*)w->col_absmax, (const uint16_t*)w->w_keep,
+                          (const int32_t*)w->keep_slot, N, K, kp > 0 ? cdiv(N, 64) : 0, wo};
             auto kern = kc <= 2 ? k_quant_rows_reg<2> : kc <= 4 ? k_quant_rows_reg<4>
                       : kc <= 6 ? k_quant_rows_reg<6> : k_quant_rows_reg<8>;
-            e = launch(kern, dim3(M), dim3(256), smem, s, true, X, M, K, (const uint32_t*)mask, max_outliers, kp,
-                       xq, ra, xo, idx, n_out, status);
+            e = launch(kern, dim3(ga.blocks + M), dim3(256), 0, s, true, X, M, K, (const uint32_t*)mask,
+                       (const int32_t*)n_out, max_outliers, kp, xq, ra, xo, (const int32_t*)idx, ga);
         } else {
             // mask words, their prefix counts, and one flag word per 2048-column window
             const size_t smem = ((size_t)cdiv(K, 32) * 2 + (size_t)cdiv(K, 2048)) * 4;
             const int grid = std::max(1, std::min(cdiv(M, 8), sms * 4));
             e = launch(k_quant_rows, dim3(grid), dim3(256), smem, s, true, X, M, K, (const uint32_t*)mask,
-                       max_outliers, kp, xq, ra, xo, idx, n_out, status);
+                       max_outliers, kp, xq, ra, xo);
+            if (e == cudaSuccess && kp > 0)
+                e = launch(k_gather_wo, dim3(cdiv(N, 64)), dim3(256), 0, s, true, (const int8_t*)w->wq,
+                           (const float*)w->col_absmax, (const uint16_t*)w->w_keep, (const int32_t*)w->keep_slot,
+                           K, N, K, (const int32_t*)idx, (const int32_t*)n_out, max_outliers, kp, wo);
         }
     }
-    if (e == cudaSuccess)
-        e = launch(k_gather_wo, dim3(cdiv(N, 64)), dim3(256), 0, s, true, (const int8_t*)w->wq,
-                   (const float*)w->col_absmax, (const uint16_t*)w->w_keep, (const int32_t*)w->keep_slot, K, N, K,
-                   (const int32_t*)idx, (const int32_t*)n_out, max_outliers, kp, wo, mask);
-    if (e == cudaSuccess) {
-        const bool pair = (path != INT8MM_PATH_GEMM_1SM) && M > kGemmBM;
+    // the GEMM over rows [r0, r0 + rows) of Xq / Xo / Y
+    auto gemm_rows = [&](int r0, int rows, bool first) -> cudaError_t {
+        const bool pair = (path != INT8MM_PATH_GEMM_1SM) && rows > kGemmBM;
+        CUtensorMap tm_a, tm_xo, tm_y;
+        int8_t* xq_r = xq + (size_t)r0 * K;
+        uint16_t* y_r = Y + (size_t)r0 * N;
+        if (!make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq_r, K, rows, K, 128, kGemmBM) ||
+            !make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, y_r, N, rows, (uint64_t)N * 2, 64, 32))
+            return cudaErrorInvalidValue;
+        if (kp > 0) {
+            if (!make_map(&tm_xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xo + (size_t)r0 * kp, kp, rows, (uint64_t)kp * 2,
+                          64, kGemmBM))
+                return cudaErrorInvalidValue;
+        } else {
+            tm_xo = tm_a;
+        }
         GemmParams p{};
-        p.M = M;
+        p.M = rows;
         p.N = N;
         p.K = K;
-        p.num_m_blocks = cdiv(M, pair ? kG2BM : kGemmBM);
+        p.num_m_blocks = cdiv(rows, pair ? kG2BM : kGemmBM);
         p.num_n_blocks = cdiv(N, pair ? kG2BN : kGemmBN);
         p.num_tiles = p.num_m_blocks * p.num_n_blocks;
         // Raster: a group of row blocks sweeps all column tiles before the next
@@ -787,42 +875,111 @@ int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w
         p.kb_int8 = cdiv(K, 128);
         p.n_outliers = n_out;
         p.cap = max_outliers;
-        p.ra = ra;
+        p.ra = ra + r0;
         p.ca = w->col_absmax;
-        p.acc_out = acc_out;
+        p.acc_out = acc_out ? acc_out + (size_t)r0 * N : nullptr;
         p.status = status;
         p.wait_limit_ns = wait_ns;
         p.test_flags = test_flags;
+        const bool pdl = !timed;
+        cudaError_t le = cudaSuccess;
         if (pair) {
             // each CTA of the pair loads 128 rows of B / Wo per slice
             CUtensorMap tm_b2, tm_wo2;
-            if (!make_map(&tm_b2, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq, K, N, K, 128, 128)) return INT8MM_ERR_CUDA;
+            if (!make_map(&tm_b2, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq, K, N, K, 128, 128))
+                return cudaErrorInvalidValue;
             if (kp > 0) {
                 if (!make_map(&tm_wo2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wo, kp, N, (uint64_t)kp * 2, 64, 128))
-                    return INT8MM_ERR_CUDA;
+                    return cudaErrorInvalidValue;
             } else {
                 tm_wo2 = tm_b2;
             }
             const int clusters = std::min(p.num_tiles, sms / 2);
             const int grid = 2 * clusters;
-            if (timed) e = cudaEventRecord(ev0, s);
-            if (e == cudaSuccess)
-                e = acc_out ? launch_ex(k_gemm_int8_2sm<true>, dim3(grid), dim3(kGemmThreads), kG2SmemBytes, s, !timed, 2,
-                                        tm_a, tm_b2, tm_xo, tm_wo2, tm_y, p)
-                            : launch_ex(k_gemm_int8_2sm<false>, dim3(grid), dim3(kGemmThreads), kG2SmemBytes, s, !timed, 2,
-                                        tm_a, tm_b2, tm_xo, tm_wo2, tm_y, p);
+            if (timed && first) le = cudaEventRecord(ev0, s);
+            if (le == cudaSuccess)
+                le = acc_out ? launch_ex(k_gemm_int8_2sm<true>, dim3(grid), dim3(kGemmThreads), kG2SmemBytes, s, pdl,
+                                         2, tm_a, tm_b2, tm_xo, tm_wo2, tm_y, p)
+                             : launch_ex(k_gemm_int8_2sm<false>, dim3(grid), dim3(kGemmThreads), kG2SmemBytes, s,
+                                         pdl, 2, tm_a, tm_b2, tm_xo, tm_wo2, tm_y, p);
         } else {
             const int grid = std::min(p.num_tiles, sms);
-            if (timed) e = cudaEventRecord(ev0, s);
-            if (e == cudaSuccess)
-                e = acc_out ? launch(k_gemm_int8_sm100<true>, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, s,
-                                     !timed, tm_a, tm_b, tm_xo, tm_wo, tm_y, p)
-                            : launch(k_gemm_int8_sm100<false>, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, s,
-                                     !timed, tm_a, tm_b, tm_xo, tm_wo, tm_y, p);
+            if (timed && first) le = cudaEventRecord(ev0, s);
+            if (le == cudaSuccess)
+                le = acc_out ? launch(k_gemm_int8_sm100<true>, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, s,
+                                      pdl, tm_a, tm_b, tm_xo, tm_wo, tm_y, p)
+                             : launch(k_gemm_int8_sm100<false>, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, s,
+                                      pdl, tm_a, tm_b, tm_xo, tm_wo, tm_y, p);
         }
+        return le;
+    };
+
+    if (!hc) {
+        if (e == cudaSuccess) e = gemm_rows(0, M, true);
         if (e == cudaSuccess && timed) e = cudaEventRecord(ev1, s);
+        return cuda_status(e);
     }
+    // host copy-back: bands of whole 256-row tiles; each band's copy waits for
+    // that band's GEMM only, and the compute stream waits for the last copy
+    const int band_rows = std::max(256, cdiv(cdiv(M, hc->bands), 256) * 256);
+    for (int r0 = 0, i = 0; e == cudaSuccess && r0 < M; r0 += band_rows, ++i) {
+        const int rows = std::min(band_rows, M - r0);
+        e = gemm_rows(r0, rows, r0 == 0);
+        if (e == cudaSuccess) e = cudaEventRecord(hc->band_done[i], s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(hc->copy, hc->band_done[i], 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(hc->y_host + (size_t)r0 * N, Y + (size_t)r0 * N, (size_t)rows * N * 2,
+                                cudaMemcpyDeviceToHost, hc->copy);
+    }
+    if (e == cudaSuccess && timed) e = cudaEventRecord(ev1, s);
+    if (e == cudaSuccess) e = cudaEventRecord(hc->copies_done, hc->copy);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hc->copies_done, 0);
     return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int8mm_status int8mm_forward_ex(const uint16_t* X, int M, const int8mm_weight* w, float threshold,
+                                int max_outliers, uint16_t* Y, void* ws, size_t ws_bytes,
+                                const int8mm_forward_opts* opts, void* stream) {
+    return forward_core(X, M, w, threshold, max_outliers, Y, ws, ws_bytes, opts, stream, nullptr);
+}
+
+int8mm_status int8mm_forward_host(const uint16_t* x_host, int M, const int8mm_weight* w, float threshold,
+                                  int max_outliers, uint16_t* y_host, uint16_t* x_dev, uint16_t* y_dev,
+                                  void* ws, size_t ws_bytes, void* stream) {
+    if (!x_host || !y_host || !x_dev || !y_dev || !w) return INT8MM_ERR_INVALID_ARGUMENT;
+    const int K = w->K, N = w->N;
+    if (!shape_ok(M, K, N)) return INT8MM_ERR_INVALID_ARGUMENT;
+    int dev;
+    DeviceInfo* info;
+    int8mm_status st = current_device(&dev, &info);
+    if (st != INT8MM_OK) return st;
+    std::lock_guard<std::mutex> lk(g_host_mu);
+    HostPipe& hp = g_host_pipe[dev];
+    if (!hp.ready) {
+        bool ok = cudaStreamCreateWithFlags(&hp.copy, cudaStreamNonBlocking) == cudaSuccess;
+        for (int i = 0; ok && i < kHostBands; ++i)
+            ok = cudaEventCreateWithFlags(&hp.band_done[i], cudaEventDisableTiming) == cudaSuccess;
+        if (ok) ok = cudaEventCreateWithFlags(&hp.copies_done, cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) {
+            cudaGetLastError();
+            return INT8MM_ERR_CUDA;
+        }
+        hp.ready = true;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // argument errors first, before anything is queued
+    {
+        const int8mm_status chk = forward_check(x_dev, M, w, threshold, max_outliers, y_dev, ws, ws_bytes);
+        if (chk != INT8MM_OK) return chk;
+    }
+    cudaError_t e = cudaMemcpyAsync(x_dev, x_host, (size_t)M * K * 2, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    HostCopy hc{y_host, hp.copy, hp.band_done, hp.copies_done, kHostBands};
+    return forward_core(x_dev, M, w, threshold, max_outliers, y_dev, ws, ws_bytes, nullptr, stream, &hc);
 }
 
 int8mm_status int8mm_forward(const uint16_t* X, int M, const int8mm_weight* w, float threshold, int max_outliers,
@@ -991,6 +1148,8 @@ int8mm_status int8mm_forward_int4(const uint16_t* X, int M, const int8mm_int4_we
     p.stages = pl.stages;
     p.xrows = pl.xrows;
     p.tmem_cols = pl.tmem_cols;
+    p.aslots = pl.aslots;
+    p.off_a = pl.off_a;
     p.off_x = pl.off_x;
     p.off_red = pl.off_red;
     p.off_bars = pl.off_bars;
@@ -1124,26 +1283,18 @@ int8mm_status int8mm_forward_grouped(const uint16_t* X, int M, const int8mm_grou
         tm_wo = tm_b;
     }
     const int sms = info->sm_count;
-    cudaError_t e;
-    {
-        const int gx = cdiv(K, 256);
-        int gy = std::max(1, std::min(cdiv(M, 8), cdiv(4 * sms, gx)));
-        int rows = cdiv(M, gy);
-        rows = (rows + 7) / 8 * 8;
-        gy = cdiv(M, rows);
-        e = launch(k_detect, dim3(gx, gy), dim3(256), 0, s, false, X, M, K, threshold, rows, mask);
-    }
+    cudaError_t e = launch_detect(X, M, K, threshold, L, b, max_outliers, s);
     if (e == cudaSuccess) {
         const size_t smem = (size_t)cdiv(K, 32) * 2 * 4;
         const long long items = (long long)M * ng;
         const int grid = (int)std::max<long long>(1, std::min<long long>(cdiv(items, 8), (long long)sms * 4));
         e = launch(k_quant_rows_grouped, dim3(grid), dim3(256), smem, s, true, X, M, K, G, (const uint32_t*)mask,
-                   max_outliers, kp, xq, ra, xo, idx, n_out, status);
+                   max_outliers, kp, xq, ra, xo);
     }
-    if (e == cudaSuccess)
+    if (e == cudaSuccess && kp > 0)
         e = launch(k_gather_wo, dim3(cdiv(N, 64)), dim3(256), 0, s, true, (const int8_t*)w->wq,
                    (const float*)w->col_absmax, (const uint16_t*)w->w_keep, (const int32_t*)w->keep_slot, K, N, G,
-                   (const int32_t*)idx, (const int32_t*)n_out, max_outliers, kp, wo, mask);
+                   (const int32_t*)idx, (const int32_t*)n_out, max_outliers, kp, wo);
     if (e == cudaSuccess) {
         GroupedParams gp{};
         GemmParams& p = gp.g;

@@ -136,14 +136,85 @@ __global__ void k_copy_keep_rows(const uint16_t* __restrict__ W, int N, const in
 
 // ------------------------------------------------------------------ (a) detect
 
+// The last block of k_detect: the bitmask as the OR of the row splits' words,
+// the exclusive prefix counts, the ascending outlier list, the count and the
+// overflow flag; resets the ticket.  All 256 threads of the block.
+__device__ __noinline__ void detect_finalise(const uint32_t* __restrict__ part, int ny, int nw,
+                                             uint32_t* __restrict__ mask, int32_t* __restrict__ spre,
+                                             int32_t* __restrict__ idx, int32_t* __restrict__ n_out, int cap,
+                                             int* __restrict__ status, unsigned* __restrict__ ticket) {
+    __shared__ int wtot[8];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    int carry = 0;
+    for (int base = 0; base < nw; base += 256) {
+        const int w = base + tid;
+        uint32_t word = 0u;
+        if (w < nw) {
+            // eight independent loads in flight per step: the splits' words
+            // come from L2, and this block's latency is on the critical path
+            int y = 0;
+            for (; y + 8 <= ny; y += 8) {
+                uint32_t t[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) t[i] = __ldcg(part + (size_t)(y + i) * nw + w);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) word |= t[i];
+            }
+            for (; y < ny; ++y) word |= __ldcg(part + (size_t)y * nw + w);
+        }
+        const int c = __popc(word);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) wtot[warp] = incl;
+        __syncthreads();
+        int before = 0, blk = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            before += i < warp ? wtot[i] : 0;
+            blk += wtot[i];
+        }
+        if (w < nw) {
+            int s = carry + before + incl - c;
+            mask[w] = word;
+            spre[w] = s;
+            while (word) {
+                idx[s++] = w * 32 + (__ffs(word) - 1);
+                word &= word - 1;
+            }
+        }
+        carry += blk;
+        __syncthreads();
+    }
+    if (tid == 0) {
+        *n_out = carry;
+        if (carry > cap) atomicOr(status, kStatusOverflow);
+        *ticket = 0u;
+    }
+}
+
 // One pass over X: column k is an outlier when max_m |X[m, k]| >= thr.
 // Block 256 threads = 8 warps over 256 columns (8 per lane); warps stride over
-// rows [row0, row1).  Flags are OR-ed into the bitmask (bit k of word k/32).
+// rows [row0, row1) of the block's row split blockIdx.y.  Each block stores
+// the 8 flag words of its columns for its row split (part[y * nw + w], bit k
+// of word k / 32; every word is written on every call, so nothing needs
+// clearing).  The last block to finish (a ticket counted in *ticket) OR-s the
+// row splits into the bitmask mask[w], forms the exclusive prefix counts
+// spre[w] (outlier columns before word w) and writes the ascending outlier
+// list idx, the count *n_out and the overflow flag, then resets the ticket.
 __global__ void __launch_bounds__(256) k_detect(const uint16_t* __restrict__ X, int M, int K, float thr,
-                                                int rows_per_block, uint32_t* __restrict__ mask) {
+                                                int rows_per_block, uint32_t* __restrict__ part,
+                                                uint32_t* __restrict__ mask, int32_t* __restrict__ spre,
+                                                int32_t* __restrict__ idx, int32_t* __restrict__ n_out, int cap,
+                                                int* __restrict__ status, unsigned* __restrict__ ticket) {
     pdl_launch_dependents();
     __shared__ uint32_t red[8][32][4];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ unsigned last_sh;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nw = (K + 31) / 32;
     const int col0 = blockIdx.x * 256 + lane * 8;
     const int row0 = blockIdx.y * rows_per_block;
     const int row1 = min(M, row0 + rows_per_block);
@@ -170,34 +241,45 @@ __global__ void __launch_bounds__(256) k_detect(const uint16_t* __restrict__ X, 
 #pragma unroll
     for (int i = 0; i < 4; ++i) red[warp][lane][i] = m[i];
     __syncthreads();
-    if (warp != 0) return;
+    if (warp == 0) {
 #pragma unroll
-    for (int w = 1; w < 8; ++w)
+        for (int w = 1; w < 8; ++w)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) m[i] = __vmaxu2(m[i], red[w][lane][i]);
-    uint32_t flags = 0;  // 8 bits, one per column of this lane
+            for (int i = 0; i < 4; ++i) m[i] = __vmaxu2(m[i], red[w][lane][i]);
+        uint32_t flags = 0;  // 8 bits, one per column of this lane
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        if (half_bits_to_float(m[i] & 0xFFFF) >= thr) flags |= 1u << (2 * i);
-        if (half_bits_to_float(m[i] >> 16) >= thr) flags |= 1u << (2 * i + 1);
+        for (int i = 0; i < 4; ++i) {
+            if (half_bits_to_float(m[i] & 0xFFFF) >= thr) flags |= 1u << (2 * i);
+            if (half_bits_to_float(m[i] >> 16) >= thr) flags |= 1u << (2 * i + 1);
+        }
+        if (col0 >= K) flags = 0;
+        // word j of this block = lanes 4j..4j+3
+        const uint32_t f1 = __shfl_down_sync(0xffffffffu, flags, 1);
+        const uint32_t f2 = __shfl_down_sync(0xffffffffu, flags, 2);
+        const uint32_t f3 = __shfl_down_sync(0xffffffffu, flags, 3);
+        const int wi = (blockIdx.x * 256 + lane * 8) >> 5;
+        if ((lane & 3) == 0 && wi < nw)
+            part[(size_t)blockIdx.y * nw + wi] = flags | (f1 << 8) | (f2 << 16) | (f3 << 24);
+        __threadfence();  // the words before the ticket
     }
-    if (col0 >= K) flags = 0;
-    // word j of this block = lanes 4j..4j+3
-    uint32_t f1 = __shfl_down_sync(0xffffffffu, flags, 1);
-    uint32_t f2 = __shfl_down_sync(0xffffffffu, flags, 2);
-    uint32_t f3 = __shfl_down_sync(0xffffffffu, flags, 3);
-    if ((lane & 3) == 0) {
-        uint32_t word = flags | (f1 << 8) | (f2 << 16) | (f3 << 24);
-        int wi = (blockIdx.x * 256 + lane * 8) >> 5;
-        if (word && wi * 32 < K) atomicOr(&mask[wi], word);
+    __syncthreads();
+    if (tid == 0) {
+        const unsigned nblk = gridDim.x * gridDim.y;
+        last_sh = (atomicAdd(ticket, 1u) == nblk - 1) ? 1u : 0u;
     }
+    __syncthreads();
+    if (!last_sh) return;
+    __threadfence();  // every block's words are visible from here on
+
+    detect_finalise(part, gridDim.y, nw, mask, spre, idx, n_out, cap, status, ticket);
 }
 
 // ------------------------------------------------------------------ (b) quantise rows
 
-// Max |x| over the non-outlier columns of one 8-column chunk c (as fp16 bits).
-__device__ __forceinline__ uint32_t chunk_inlier_absmax(uint4 v, const uint32_t* smask, int c) {
-    const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;  // outlier flags of columns 8c..8c+7
+// Max |x| over the non-outlier columns of one 8-column chunk (as fp16 bits);
+// fl = the chunk's 8 outlier flags (bit j: column j of the chunk).  Taken only
+// by chunks that hold an outlier column, so it is kept out of line.
+__device__ __noinline__ uint32_t chunk_inlier_absmax(uint4 v, uint32_t fl) {
     const uint32_t h[4] = {v.x, v.y, v.z, v.w};
     uint32_t amax = 0;
 #pragma unroll
@@ -251,10 +333,12 @@ __device__ __forceinline__ uint32_t chunk_absmax_h2(uint4 v) {
 
 
 // Quantise one 8-column chunk c of a row; outlier columns give 0 and are
-// copied to their slot of the row's fp16 outlier vector.
-__device__ __forceinline__ uint2 quant_chunk(uint4 v, const uint32_t* smask, const int* spre, int c, float rmax,
-                                            float scale, int n_eff, uint16_t* xo_row) {
-    const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
+// copied to their slot of the row's fp16 outlier vector.  word = the mask word
+// holding the chunk (columns 32 * (c / 4) ...), pre = the outlier columns
+// before that word.  Taken only by chunks that hold an outlier column.
+__device__ __noinline__ uint2 quant_chunk(uint4 v, uint32_t word, int pre, int c, float rmax, float scale,
+                                          int n_eff, uint16_t* xo_row) {
+    const uint32_t fl = (word >> ((c & 3) * 8)) & 0xFFu;
     const uint32_t h[4] = {v.x, v.y, v.z, v.w};
     uint32_t out[2] = {0u, 0u};
 #pragma unroll
@@ -265,8 +349,7 @@ __device__ __forceinline__ uint2 quant_chunk(uint4 v, const uint32_t* smask, con
             if (rmax > 0.0f) q = quant1(half_bits_to_float(bits), scale);
         } else {
             const int k = c * 8 + j;
-            const int w = k >> 5;
-            const int slot = spre[w] + __popc(smask[w] & ((1u << (k & 31)) - 1u));
+            const int slot = pre + __popc(word & ((1u << (k & 31)) - 1u));
             if (slot < n_eff) xo_row[slot] = (uint16_t)bits;
         }
         out[j >> 2] |= ((uint32_t)(q & 0xFF)) << ((j & 3) * 8);
@@ -306,31 +389,10 @@ __device__ __forceinline__ int load_mask_prefix(const uint32_t* __restrict__ mas
     return carry;
 }
 
-// Block 0's part of the row quantisers: the outlier count, the overflow flag
-// and the ascending outlier list.
-__device__ __forceinline__ void write_outlier_list(const uint32_t* smask, const int* spre, int nw, int total, int cap,
-                                                   int32_t* __restrict__ idx, int32_t* __restrict__ n_out,
-                                                   int* __restrict__ status) {
-    const int tid = threadIdx.x;
-    if (tid == 0) {
-        *n_out = total;
-        if (total > cap) atomicOr(status, kStatusOverflow);
-    }
-    for (int w = tid; w < nw; w += 256) {
-        uint32_t word = smask[w];
-        int s = spre[w];
-        while (word) {
-            const int b = __ffs(word) - 1;
-            idx[s++] = w * 32 + b;
-            word &= word - 1;
-        }
-    }
-}
-
 // Per row m: ra[m] = max over non-outlier columns of |X[m,k]|,
 // Xq[m,k] = outlier ? 0 : q(X[m,k]), Xo[m, slot(k)] = X[m,k] for outlier k,
-// with Xo zero-padded to a multiple of 64 columns.  Block 0 also writes the
-// ascending outlier list, the count and the overflow flag.
+// with Xo zero-padded to a multiple of 64 columns (the outlier list, count
+// and overflow flag come from k_detect).
 // One warp per row (no block barrier inside the row loop): a first pass over
 // the row takes the absmax with 8 independent 16-byte loads in flight per
 // lane, a second pass (served by L1/L2) writes the codes.  Block: 256 threads
@@ -338,8 +400,7 @@ __device__ __forceinline__ void write_outlier_list(const uint32_t* smask, const 
 __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__ X, int M, int K,
                                                     const uint32_t* __restrict__ mask, int cap, int kp,
                                                     int8_t* __restrict__ Xq, float* __restrict__ ra,
-                                                    uint16_t* __restrict__ Xo, int32_t* __restrict__ idx,
-                                                    int32_t* __restrict__ n_out, int* __restrict__ status) {
+                                                    uint16_t* __restrict__ Xo) {
     extern __shared__ uint32_t qsm[];
     const int nw = (K + 31) / 32;
     uint32_t* smask = qsm;                          // nw words
@@ -369,8 +430,6 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
     const int n_eff = min(total, cap);
     const int n_pad = min(kp, (n_eff + 63) / 64 * 64);
 
-    if (blockIdx.x == 0) write_outlier_list(smask, spre, nw, total, cap, idx, n_out, status);
-
     for (int m = blockIdx.x * 8 + warp; m < M; m += gridDim.x * 8) {
         const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)m * K);
         uint32_t amax = 0;
@@ -391,7 +450,7 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
                 const int c = c0 + 32 * i;
                 if (c < nchunk) {
                     const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
-                    amax = max(amax, fl ? chunk_inlier_absmax(v[i], smask, c) : chunk_absmax_h2(v[i]));
+                    amax = max(amax, fl ? chunk_inlier_absmax(v[i], fl) : chunk_absmax_h2(v[i]));
                 }
             }
         }
@@ -418,7 +477,8 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
                 const int c = c0 + 32 * i;
                 if (c < nchunk) {
                     const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
-                    qr[c] = fl ? quant_chunk(v[i], smask, spre, c, rmax, scale, n_eff, xo_row) : quant8_plain(v[i], scale);
+                    qr[c] = fl ? quant_chunk(v[i], smask[c >> 2], spre[c >> 2], c, rmax, scale, n_eff, xo_row)
+                               : quant8_plain(v[i], scale);
                 }
             }
         }
@@ -426,108 +486,16 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
     }
 }
 
-// k_quant_rows with one row per 256-thread block, the row held in registers
-// (kC 8-column chunks per thread, K <= 2048 * kC), so X is read from memory
-// once.  The row's loads go out first; the block copies the outlier bitmask to
-// shared memory (barrier 1); warp 0 then forms the words' prefix counts while
-// every warp takes its part of the row maximum over the non-outlier columns,
-// and one more barrier (2) publishes both; the codes and the outlier values
-// follow in the same pass (each warp stores 256 contiguous bytes per step).
-// Block 0 also writes the outlier list, the count and the overflow flag.  Same
-// results as k_quant_rows.
-template <int kC>
-__global__ void __launch_bounds__(256) k_quant_rows_reg(const uint16_t* __restrict__ X, int M, int K,
-                                                        const uint32_t* __restrict__ mask, int cap, int kp,
-                                                        int8_t* __restrict__ Xq, float* __restrict__ ra,
-                                                        uint16_t* __restrict__ Xo, int32_t* __restrict__ idx,
-                                                        int32_t* __restrict__ n_out, int* __restrict__ status) {
-    extern __shared__ uint32_t qsm[];
-    const int nw = (K + 31) / 32;
-    uint32_t* smask = qsm;
-    int* spre = reinterpret_cast<int*>(qsm + nw);
-    __shared__ uint32_t bmax[8];
-    __shared__ int total_sh;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int m = blockIdx.x;
-    const int nchunk = K / 8;
-
-    pdl_wait();  // the outlier bitmask comes from k_detect
-    pdl_launch_dependents();
-    const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)m * K);
-    uint4 v[kC];
-#pragma unroll
-    for (int i = 0; i < kC; ++i) {
-        const int c = tid + 256 * i;
-        if (c < nchunk) v[i] = __ldg(xr + c);
-    }
-    for (int w = tid; w < nw; w += 256) smask[w] = __ldg(mask + w);
-    __syncthreads();  // (1) the bitmask
-    if (warp == 0) {
-        // exclusive prefix counts of the words, lane l taking words [l*per, (l+1)*per)
-        const int per = (nw + 31) / 32;
-        const int w0 = min(nw, lane * per), w1 = min(nw, w0 + per);
-        int cnt = 0;
-        for (int w = w0; w < w1; ++w) cnt += __popc(smask[w]);
-        int incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += t;
-        }
-        int run = incl - cnt;
-        for (int w = w0; w < w1; ++w) {
-            spre[w] = run;
-            run += __popc(smask[w]);
-        }
-        if (lane == 31) total_sh = incl;
-    }
-    uint32_t amax = 0;
-#pragma unroll
-    for (int i = 0; i < kC; ++i) {
-        const int c = tid + 256 * i;
-        if (c < nchunk) {
-            const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
-            amax = max(amax, fl ? chunk_inlier_absmax(v[i], smask, c) : chunk_absmax_h2(v[i]));
-        }
-    }
-    amax = __reduce_max_sync(0xffffffffu, amax);
-    if (lane == 0) bmax[warp] = amax;
-    __syncthreads();  // (2) the prefix counts, the total and the warps' maxima
-    const int total = total_sh;
-    const int n_eff = min(total, cap);
-    const int n_pad = min(kp, (n_eff + 63) / 64 * 64);
-    if (m == 0) write_outlier_list(smask, spre, nw, total, cap, idx, n_out, status);
-    amax = 0;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) amax = max(amax, bmax[w]);
-    const float rmax = half_bits_to_float(amax);
-    const float scale = rmax > 0.0f ? __fdiv_rn(127.0f, rmax) : 0.0f;
-    if (tid == 0) ra[m] = rmax;
-    uint2* qr = reinterpret_cast<uint2*>(Xq + (size_t)m * K);
-    uint16_t* xo_row = Xo + (size_t)m * kp;
-#pragma unroll
-    for (int i = 0; i < kC; ++i) {
-        const int c = tid + 256 * i;
-        if (c < nchunk) {
-            const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
-            qr[c] = fl ? quant_chunk(v[i], smask, spre, c, rmax, scale, n_eff, xo_row) : quant8_plain(v[i], scale);
-        }
-    }
-    for (int j = n_eff + tid; j < n_pad; j += 256) xo_row[j] = 0;
-}
-
 // Group-wise variant of k_quant_rows: one constant per row and group of G
 // consecutive columns (G a multiple of 128), ra[m * (K/G) + g] = max |X[m,k]|
 // over the non-outlier columns of the group, and the codes of the group
 // with its own scale.  One warp per (row, group) item, lanes strided over the
 // group's 8-column chunks: a first pass takes the maximum, a second (served
-// by L1/L2) writes the codes and the outlier values.  Block 0 also writes the
-// outlier list, the count and the overflow flag.  Block 256 threads.
+// by L1/L2) writes the codes and the outlier values.  Block 256 threads.
 __global__ void __launch_bounds__(256) k_quant_rows_grouped(const uint16_t* __restrict__ X, int M, int K, int G,
                                                             const uint32_t* __restrict__ mask, int cap, int kp,
                                                             int8_t* __restrict__ Xq, float* __restrict__ ra,
-                                                            uint16_t* __restrict__ Xo, int32_t* __restrict__ idx,
-                                                            int32_t* __restrict__ n_out, int* __restrict__ status) {
+                                                            uint16_t* __restrict__ Xo) {
     extern __shared__ uint32_t qsm[];
     const int nw = (K + 31) / 32;
     uint32_t* smask = qsm;
@@ -540,8 +508,6 @@ __global__ void __launch_bounds__(256) k_quant_rows_grouped(const uint16_t* __re
     const int total = load_mask_prefix(mask, nw, smask, spre, red);
     const int n_eff = min(total, cap);
     const int n_pad = min(kp, (n_eff + 63) / 64 * 64);
-    if (blockIdx.x == 0) write_outlier_list(smask, spre, nw, total, cap, idx, n_out, status);
-
     const int ng = K / G, cpg = G / 8;  // chunks per group
     const long long items = (long long)M * ng;
     for (long long it = (long long)blockIdx.x * 8 + warp; it < items; it += (long long)gridDim.x * 8) {
@@ -552,7 +518,7 @@ __global__ void __launch_bounds__(256) k_quant_rows_grouped(const uint16_t* __re
         for (int c = c0 + lane; c < c1; c += 32) {
             const uint4 v = __ldg(xr + c);
             const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
-            amax = max(amax, fl ? chunk_inlier_absmax(v, smask, c) : chunk_absmax_h2(v));
+            amax = max(amax, fl ? chunk_inlier_absmax(v, fl) : chunk_absmax_h2(v));
         }
         amax = __reduce_max_sync(0xffffffffu, amax);
         const float rmax = half_bits_to_float(amax);
@@ -563,7 +529,8 @@ __global__ void __launch_bounds__(256) k_quant_rows_grouped(const uint16_t* __re
         for (int c = c0 + lane; c < c1; c += 32) {
             const uint4 v = __ldg(xr + c);
             const uint32_t fl = (smask[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
-            qr[c] = fl ? quant_chunk(v, smask, spre, c, rmax, scale, n_eff, xo_row) : quant8_plain(v, scale);
+            qr[c] = fl ? quant_chunk(v, smask[c >> 2], spre[c >> 2], c, rmax, scale, n_eff, xo_row)
+                       : quant8_plain(v, scale);
         }
         if (g == 0)
             for (int j = n_eff + lane; j < n_pad; j += 32) xo_row[j] = 0;
@@ -576,45 +543,40 @@ __global__ void __launch_bounds__(256) k_quant_rows_grouped(const uint16_t* __re
 // row W[idx[j], n] when idx[j] was kept at preparation, else the dequantised
 // value fp16(Wq[n, idx[j]] * ca / 127) with the constant of column n and of
 // the group of idx[j] (ca[(k / G) * N + n]; G = K: one per column); zero for
-// n_eff <= j < pad64(n_eff).
-// Block 256 threads over 64 output channels; block 0 clears the outlier
-// bitmask for the next call.
-__global__ void __launch_bounds__(256) k_gather_wo(const int8_t* __restrict__ Wq, const float* __restrict__ ca,
-                                                   const uint16_t* __restrict__ w_keep,
-                                                   const int32_t* __restrict__ keep_slot, int K, int N, int G,
-                                                   const int32_t* __restrict__ idx,
-                                                   const int32_t* __restrict__ n_out, int cap, int kp,
-                                                   uint16_t* __restrict__ Wo, uint32_t* __restrict__ mask) {
-    __shared__ uint16_t tile[64][64 + 8];
+// n_eff <= j < pad64(n_eff).  One 256-thread block builds the 64 output
+// channels from n0: a 64 x 64 tile per 64 outliers, filled along n and
+// written along j (row stride 66 halves, so the column reads of the write-out
+// meet at most two to a bank).
+__device__ __forceinline__ void gather_wo_tile(int n0, const int8_t* __restrict__ Wq, const float* __restrict__ ca,
+                                               const uint16_t* __restrict__ w_keep,
+                                               const int32_t* __restrict__ keep_slot, int K, int N, int G,
+                                               const int32_t* __restrict__ idx, const int32_t* __restrict__ n_out,
+                                               int cap, int kp, uint16_t* __restrict__ Wo) {
+    __shared__ uint16_t tile[64][66];
     __shared__ int sidx[64];
     __shared__ int sslot[64];
-    pdl_wait();
-    pdl_launch_dependents();
     const int tid = threadIdx.x;
-    if (blockIdx.x == 0)
-        for (int w = tid; w < (K + 31) / 32; w += 256) mask[w] = 0u;
-    const int n_eff = min(*n_out, cap);
+    const int n_eff = min(__ldg(n_out), cap);
     const int n_pad = min(kp, (n_eff + 63) / 64 * 64);
-    const int n0 = blockIdx.x * 64;
     for (int j0 = 0; j0 < n_pad; j0 += 64) {
         __syncthreads();
         if (tid < 64) {
-            int j = j0 + tid;
-            int k = j < n_eff ? idx[j] : -1;
+            const int j = j0 + tid;
+            const int k = j < n_eff ? __ldg(idx + j) : -1;
             sidx[tid] = k;
-            sslot[tid] = k >= 0 ? keep_slot[k] : -1;
+            sslot[tid] = k >= 0 ? __ldg(keep_slot + k) : -1;
         }
         __syncthreads();
         // fill tile[j][n]: coalesced along n
         for (int e = tid; e < 64 * 64; e += 256) {
-            int jl = e >> 6, nl = e & 63;
-            int n = n0 + nl, k = sidx[jl], slot = sslot[jl];
+            const int jl = e >> 6, nl = e & 63;
+            const int n = n0 + nl, k = sidx[jl], slot = sslot[jl];
             uint16_t v = 0;
             if (k >= 0 && n < N) {
                 if (slot >= 0) {
-                    v = w_keep[(size_t)slot * N + n];
+                    v = __ldg(w_keep + (size_t)slot * N + n);
                 } else {
-                    float t = __fmul_rn((float)Wq[(size_t)n * K + k], ca[(size_t)(k / G) * N + n]);
+                    const float t = __fmul_rn((float)Wq[(size_t)n * K + k], ca[(size_t)(k / G) * N + n]);
                     v = __half_as_ushort(__float2half_rn(__fdiv_rn(t, 127.0f)));
                 }
             }
@@ -623,8 +585,8 @@ __global__ void __launch_bounds__(256) k_gather_wo(const int8_t* __restrict__ Wq
         __syncthreads();
         // write Wo[n][j0 .. j0+64): 64 rows x 128 bytes, 8 threads per row
         for (int e = tid; e < 64 * 8; e += 256) {
-            int nl = e >> 3, c = (e & 7) * 8;
-            int n = n0 + nl;
+            const int nl = e >> 3, c = (e & 7) * 8;
+            const int n = n0 + nl;
             if (n >= N) continue;
             uint32_t w4[4];
 #pragma unroll
@@ -633,6 +595,141 @@ __global__ void __launch_bounds__(256) k_gather_wo(const int8_t* __restrict__ Wq
             *reinterpret_cast<uint4*>(Wo + (size_t)n * kp + j0 + c) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
     }
+}
+
+// The gather as a kernel of its own (the paths whose row quantiser is not
+// k_quant_rows_reg): block b builds channels [64 b, 64 b + 64).
+__global__ void __launch_bounds__(256) k_gather_wo(const int8_t* __restrict__ Wq, const float* __restrict__ ca,
+                                                   const uint16_t* __restrict__ w_keep,
+                                                   const int32_t* __restrict__ keep_slot, int K, int N, int G,
+                                                   const int32_t* __restrict__ idx,
+                                                   const int32_t* __restrict__ n_out, int cap, int kp,
+                                                   uint16_t* __restrict__ Wo) {
+    pdl_wait();
+    pdl_launch_dependents();
+    gather_wo_tile(blockIdx.x * 64, Wq, ca, w_keep, keep_slot, K, N, G, idx, n_out, cap, kp, Wo);
+}
+
+// Max |x| (fp16 bits) of an 8-column chunk over its non-outlier columns, fl
+// = the chunk's 8 outlier flags; branch-free (the outlier halves are cleared
+// before the native half2 max, which, as in chunk_absmax_h2, ignores NaN).
+__device__ __forceinline__ uint32_t chunk_absmax_masked(uint4 v, uint32_t fl) {
+    const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+    __half2 a[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t keep = (((fl >> (2 * j)) & 1u) ? 0u : 0x0000FFFFu) | (((fl >> (2 * j + 1)) & 1u) ? 0u : 0xFFFF0000u);
+        const uint32_t b = h[j] & 0x7FFF7FFFu & keep;
+        memcpy(&a[j], &b, 4);
+    }
+    const __half2 zero = __floats2half2_rn(0.0f, 0.0f);
+    const __half2 m = __hmax2(zero, __hmax2(__hmax2(a[0], a[1]), __hmax2(a[2], a[3])));
+    uint32_t mb;
+    memcpy(&mb, &m, 4);
+    return max(mb & 0xFFFFu, mb >> 16);
+}
+
+// 0xFF in byte j of the result for every set bit j < 4 of f.
+__device__ __forceinline__ uint32_t spread_bits_to_bytes(uint32_t f) {
+    return ((f & 0xFu) * 0x00204081u & 0x01010101u) * 0xFFu;
+}
+
+// Gather arguments of the fused register quantiser (see gather_wo_tile).
+struct GatherArgs {
+    const int8_t* Wq;
+    const float* ca;
+    const uint16_t* w_keep;
+    const int32_t* keep_slot;
+    int N, G, blocks;  // blocks = ceil(N / 64) gather tiles in front of the rows
+    uint16_t* Wo;
+};
+
+// k_quant_rows with one row per 256-thread block, the row held in registers
+// (kC 8-column chunks per thread, K <= 2048 * kC), so X is read from memory
+// once: the row's 16-byte loads and its outlier flag words (the bitmask that
+// k_detect finalised, read through L1) go out together, every warp takes its
+// part of the row maximum over the non-outlier columns, one barrier joins the
+// warps' maxima, and the codes follow in the same pass (each warp stores 256
+// contiguous bytes per step); the row's fp16 outlier values are then copied
+// by the outlier list.  The first ga.blocks blocks of the grid instead build
+// 64-channel tiles of the outlier weight rows (gather_wo_tile), which need
+// only k_detect's list, so that work runs beside the rows rather than after
+// them.  Same results as k_quant_rows.
+template <int kC>
+__global__ void __launch_bounds__(256) k_quant_rows_reg(const uint16_t* __restrict__ X, int M, int K,
+                                                        const uint32_t* __restrict__ mask,
+                                                        const int32_t* __restrict__ n_out, int cap, int kp,
+                                                        int8_t* __restrict__ Xq, float* __restrict__ ra,
+                                                        uint16_t* __restrict__ Xo, const int32_t* __restrict__ idx,
+                                                        GatherArgs ga) {
+    __shared__ uint32_t bmax[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nchunk = K / 8;
+
+    pdl_wait();  // mask, prefix counts, list and count come from k_detect
+    pdl_launch_dependents();
+    if ((int)blockIdx.x < ga.blocks) {
+        gather_wo_tile(blockIdx.x * 64, ga.Wq, ga.ca, ga.w_keep, ga.keep_slot, K, ga.N, ga.G, idx, n_out, cap, kp,
+                       ga.Wo);
+        return;
+    }
+    const int m = blockIdx.x - ga.blocks;
+    const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)m * K);
+    uint4 v[kC];
+    uint32_t fl[kC];  // the outlier flags of each chunk's 8 columns
+#pragma unroll
+    for (int i = 0; i < kC; ++i) {
+        const int c = tid + 256 * i;
+        fl[i] = 0u;
+        if (c < nchunk) {
+            v[i] = __ldg(xr + c);
+            fl[i] = (__ldg(mask + (c >> 2)) >> ((c & 3) * 8)) & 0xFFu;
+        }
+    }
+    const int n_eff = min(__ldg(n_out), cap);
+    // Chunks with an outlier column are rare (a few per row); a warp that
+    // holds one takes the masked forms for that step, all lanes together.
+    // The votes are taken by every lane of the warp (fl is 0 past the row).
+    uint32_t any_fl = 0u;  // bit i: some lane of the warp has an outlier column in step i
+#pragma unroll
+    for (int i = 0; i < kC; ++i) any_fl |= (__any_sync(0xffffffffu, fl[i] != 0u) ? 1u : 0u) << i;
+    uint32_t amax = 0;
+#pragma unroll
+    for (int i = 0; i < kC; ++i) {
+        const int c = tid + 256 * i;
+        if (c < nchunk)
+            amax = max(amax, ((any_fl >> i) & 1u) ? chunk_absmax_masked(v[i], fl[i]) : chunk_absmax_h2(v[i]));
+    }
+    amax = __reduce_max_sync(0xffffffffu, amax);
+    if (lane == 0) bmax[warp] = amax;
+    __syncthreads();  // the warps' maxima
+    amax = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) amax = max(amax, bmax[w]);
+    const float rmax = half_bits_to_float(amax);
+    const float scale = rmax > 0.0f ? __fdiv_rn(127.0f, rmax) : 0.0f;
+    if (tid == 0) ra[m] = rmax;
+    uint2* qr = reinterpret_cast<uint2*>(Xq + (size_t)m * K);
+#pragma unroll
+    for (int i = 0; i < kC; ++i) {
+        const int c = tid + 256 * i;
+        if (c < nchunk) {
+            uint2 q = quant8_plain(v[i], scale);
+            // outlier columns get code 0 (their products go through fp16); the
+            // other codes of the chunk are exact as they stand, since those
+            // columns are bounded by the row maximum
+            if ((any_fl >> i) & 1u) {
+                q.x &= ~spread_bits_to_bytes(fl[i]);
+                q.y &= ~spread_bits_to_bytes(fl[i] >> 4);
+            }
+            qr[c] = q;
+        }
+    }
+    // the row's fp16 outlier values by the list (the row is in L1), zero-padded
+    uint16_t* xo_row = Xo + (size_t)m * kp;
+    const int n_pad = min(kp, (n_eff + 63) / 64 * 64);
+    for (int j = tid; j < n_pad; j += 256)
+        xo_row[j] = j < n_eff ? __ldg(X + (size_t)m * K + __ldg(idx + j)) : (uint16_t)0;
 }
 
 }  // namespace i8mm
