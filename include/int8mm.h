@@ -312,7 +312,7 @@ int8mm_status int8mm_prepare_weight_int4(const uint16_t* W, int K, int N, int G,
  * 1 <= M <= 16:  y[m,n] = sum_k x[m,k] * (q[n,k] * absmax[n,g(k)] / 7), the
  * products on the tensor cores with fp32 sums, rounded to fp16 once.
  * The kernel keeps its share of X in shared memory, which bounds K: K <=
- * 40960 for M <= 8 and K <= 12288 for 9 <= M <= 16; longer K returns
+ * 73728 for M <= 8 and K <= 28672 for 9 <= M <= 16; longer K returns
  * INT8MM_ERR_INVALID_ARGUMENT.
  * status: device int32 word, zero before the call; a wait in the kernel that
  * runs out sets bit 0 (INT8MM_ERR_TIMEOUT: outputs invalid).  Stream-ordered

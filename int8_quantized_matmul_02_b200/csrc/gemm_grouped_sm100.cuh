@@ -61,6 +61,15 @@ constexpr int kGGSmemBytes =
     1024 + kGGStages * kGGStageBytes + kGGEpiWarps * (2 * kGemmEpiBufBytes + kGGCaBytes) + 256;
 constexpr uint32_t kGGSumCol = 256;                // running fp32 sums; accumulators at 0 and 128
 
+// Arrive on a barrier of a CTA in the cluster without release semantics.  Used
+// where the arrival only says that this thread's tensor-memory loads have
+// completed (tcgen05.wait::ld, then tcgen05.fence::before_thread_sync): no
+// ordinary memory write has to become visible with it, and a release would
+// wait for this thread's outstanding loads of global memory.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+
 // Pairs of fp32 lanes in one instruction (sm_100 packed f32x2 arithmetic;
 // each lane rounds as its scalar counterpart does).
 __device__ __forceinline__ void mul2_rn(float& d0, float& d1, float a0, float a1, float b) {
@@ -330,9 +339,9 @@ __global__ void __launch_bounds__(kGGThreads, 1)
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
-                // the accumulator is free; the release is issued before the next
-                // group's constant loads so that it does not wait for them
-                if (lane == 0) mbar_arrive_cluster(tempty_even[acc]);
+                // the accumulator is free (issued before the next group's
+                // constant loads)
+                if (lane == 0) mbar_arrive_cluster_relaxed(tempty_even[acc]);
                 if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1;

@@ -30,15 +30,15 @@
 // Forward kernel: clusters of CL CTAs split K (CTA r owns the r-th K range of
 // the cluster's tiles of 128 output columns) as the 8-bit decode kernel
 // does; warp 0 streams 128 (columns) x 256 (k) boxes of packed codes through a
-// TMA ring from launch on, warps 2-5 widen each half box (128 k) to fp16 and
-// write it to shared memory as the A operand, in the K-major 128-byte
-// swizzled layout that the MMA reads (thread = output column = row of A;
-// three such operands in flight), warp 1 issues tcgen05.mma kind::f16 with A
+// TMA ring from launch on, warps 2-9 widen each half box (128 k) to fp16 and
+// write it to tensor memory as the A operand (thread = output column =
+// TMEM lane, two warps per lane quarter, one per 64 k; four such operands in
+// flight), warp 1 issues tcgen05.mma kind::f16 with A from tensor memory
 // and X (loaded once by TMA, 128-byte swizzled, K-major) as the 16-column B
-// operand from shared memory into one of four fp32 accumulators in tensor
-// memory (an A operand in tensor memory instead takes more than twice the
-// issue time per MMA at this N), and warps 6-9 drain each
-// accumulator, scale it and add it up per column; the partial sums of a
+// operand into one of sixteen fp32 accumulators, and warps 10-13 drain them
+// four at a time (one wait and one 64-column load per four 128-k blocks, so
+// that the drain's latency is paid once per four blocks), scale each by its
+// group's constant and add them up per column; the partial sums of a
 // tile then go to the tile's owner in the cluster (asynchronous stores into
 // its shared memory), which adds them in a fixed order and writes fp16 Y.
 #pragma once
@@ -101,20 +101,32 @@ struct Int4Params {
     int M, K, N, G;
     int num_tiles, kb_total;    // 128-column tiles, 256-k boxes
     int num_clusters, cluster, stages, xrows;  // xrows: rows of one X box (8 or 16)
-    int aslots;                 // A operands in flight (2 or 3)
     uint32_t tmem_cols;
-    uint32_t off_a, off_x, off_red, off_bars;  // shared-memory offsets
+    uint32_t off_x, off_red, off_bars;  // shared-memory offsets
 };
 
-constexpr int kI4Threads = 320;          // warp 0 TMA, 1 MMA, 2-5 widen, 6-9 accumulate
+constexpr int kI4Threads = 448;          // warp 0 TMA, 1 MMA, 2-9 widen, 10-13 accumulate
+constexpr int kI4WidenWarps = 8;
 constexpr int kI4TileN = 128;
 constexpr int kI4BoxK = 256;             // k per packed box (128 bytes per row)
 constexpr int kI4StageBytes = kI4TileN * 128;  // 16 KB
-constexpr int kI4DSlots = 4;             // fp32 accumulators in TMEM (16 columns each)
-constexpr int kI4ASlots = 3;             // at most this many fp16 A operands in shared memory (128 rows x 128 k)
-constexpr int kI4ABytes = kI4TileN * 128 * 2;  // 32 KB: two 16 KB K-major 128-byte-swizzled halves of 64 k
-constexpr uint32_t kI4DColBase = 0;
-constexpr uint32_t kI4TmemCols = 64;     // the four accumulators
+constexpr int kI4DSlots = 16;            // fp32 accumulators in TMEM (16 columns each)
+constexpr int kI4DBatch = 4;             // accumulators drained per wait (64 columns, one load pair)
+constexpr int kI4ASlots = 4;             // fp16 A operands in TMEM (64 columns = 128 k each)
+constexpr uint32_t kI4AColBase = 0;
+constexpr uint32_t kI4DColBase = 64 * kI4ASlots;
+constexpr uint32_t kI4TmemCols = 512;    // the whole TMEM of the SM: one CTA per SM
+
+__device__ __forceinline__ void i4_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+    const uint32_t z = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(z)
+        : "memory");
+}
 
 // fp16 pairs of the 8 codes in one packed word (see the layout above)
 __device__ __forceinline__ void i4_widen(uint32_t w, uint32_t* out) {
@@ -135,7 +147,6 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = smem;
-    uint8_t* sa = smem + p.off_a;  // [p.aslots] fp16 A operands
     uint8_t* sx = smem + p.off_x;
     float* sred = reinterpret_cast<float*>(smem + p.off_red);  // [CL][128][RS] peers' partial sums, then its own
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bars);
@@ -144,7 +155,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     uint64_t* afull = bars + 2 * p.stages;  // [kI4ASlots]
     uint64_t* afree = afull + kI4ASlots;    // [kI4ASlots]
     uint64_t* dfull = afree + kI4ASlots;    // [kI4DSlots]
-    uint64_t* dfree = dfull + kI4DSlots;    // [4]
+    uint64_t* dfree = dfull + kI4DSlots;    // [kI4DSlots]
     uint64_t* xfull = dfree + kI4DSlots;
     uint64_t* red_done = xfull + 1;
     uint64_t* drain = xfull + 2;
@@ -174,10 +185,10 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         if (lane == 0) {
             for (int s = 0; s < p.stages; ++s) {
                 mbar_init(&full[s], 1);
-                mbar_init(&empty[s], 4);
+                mbar_init(&empty[s], kI4WidenWarps);
             }
             for (int a = 0; a < kI4ASlots; ++a) {
-                mbar_init(&afull[a], 4);
+                mbar_init(&afull[a], kI4WidenWarps);
                 mbar_init(&afree[a], 1);
             }
             for (int d = 0; d < kI4DSlots; ++d) {
@@ -244,8 +255,8 @@ __global__ void __launch_bounds__(kI4Threads, 1)
             bool ok = wait_bounded_sleep(xfull, 0, wctx), issued = false;
             tc_fence_after();
             for (int i = 0; ok && i < nb; ++i) {
-                const int a = i % p.aslots, d = i % kI4DSlots;
-                if (!wait_bounded_sleep(&afull[a], (uint32_t)((i / p.aslots) & 1), wctx) ||
+                const int a = i % kI4ASlots, d = i % kI4DSlots;
+                if (!wait_bounded_sleep(&afull[a], (uint32_t)((i / kI4ASlots) & 1), wctx) ||
                     !wait_bounded_sleep(&dfree[d], (uint32_t)(((i / kI4DSlots) & 1) ^ 1), wctx)) {
                     ok = false;
                     break;
@@ -253,15 +264,13 @@ __global__ void __launch_bounds__(kI4Threads, 1)
                 tc_fence_after();
                 const int b = i % nblk;  // 128-k block within the K range
                 const uint32_t dt = tmem_base + kI4DColBase + 16u * (uint32_t)d;
-                const uint32_t a0 = smem_u32(sa + (size_t)a * kI4ABytes);
+                const uint32_t at = tmem_base + kI4AColBase + 64u * (uint32_t)a;
 #pragma unroll
                 for (int st = 0; st < 8; ++st) {
-                    // A: half st / 4 of the operand, 32-byte step (st % 4) inside its rows;
                     // B: k = b * 128 + 16 st within the range -> X box (k / 64), 32-byte step inside it
-                    const uint64_t da = sdesc_k128sw(a0 + (uint32_t)(st >> 2) * (kI4ABytes / 2)) + (uint64_t)(2 * (st & 3));
                     const int kk = b * 128 + 16 * st;
                     const uint64_t db = db0 + (uint64_t)(((uint32_t)(kk >> 6) * xbox_bytes + (uint32_t)((kk & 63) * 2)) >> 4);
-                    mma_f16(dt, da, db, idesc, st > 0 ? 1u : 0u);
+                    i4_mma_f16_ts(dt, at + 8u * (uint32_t)st, db, idesc, st > 0 ? 1u : 0u);
                 }
                 tc_commit(&afree[a]);
                 tc_commit(&dfull[d]);
@@ -272,37 +281,35 @@ __global__ void __launch_bounds__(kI4Threads, 1)
                 wait_drain(drain, 0, 50ull * 1000 * 1000);
             }
         }
-    } else if (warp < 6) {
-        // ------------------------------------------------ widen codes to fp16 A operands in shared memory
+    } else if (warp < 2 + kI4WidenWarps) {
+        // ------------------------------------------------ widen codes to fp16 A operands in TMEM
         const int quad = warp & 3;
-        const int row = quad * 32 + lane;  // output column within the tile = row of A
+        const int part = (warp - 2) >> 2;  // this warp's 64 k of each 128-k block
+        const int row = quad * 32 + lane;  // output column within the tile = TMEM lane
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         bool ok = true;
         for (int i = 0; ok && i < nb; ++i) {
-            const int t = i >> 1, h = i & 1, a = i % p.aslots;
+            const int t = i >> 1, h = i & 1, a = i % kI4ASlots;
             const int stage = t % p.stages;
             const uint32_t ph = (uint32_t)((t / p.stages) & 1);
             ok = __all_sync(0xffffffffu, wait_bounded_sleep(&full[stage], ph, wctx)) &&
-                 __all_sync(0xffffffffu, wait_bounded_sleep(&afree[a], (uint32_t)(((i / p.aslots) & 1) ^ 1), wctx));
+                 __all_sync(0xffffffffu, wait_bounded_sleep(&afree[a], (uint32_t)(((i / kI4ASlots) & 1) ^ 1), wctx));
             if (!ok) break;
+            tc_fence_after();
             const uint8_t* src = ring + stage * kI4StageBytes + row * 128;
-            uint8_t* dst = sa + (size_t)a * kI4ABytes + row * 128;
+            uint32_t v[32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                // packed 16-byte chunk 4h + c of the row (128-byte swizzle) = 32 k = four fp16 chunks
-                const int cs = 4 * h + c;
-                const uint4 w = *reinterpret_cast<const uint4*>(src + ((cs ^ (row & 7)) << 4));
-                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    // fp16 chunk q = 4c + u (8 k) of the 128-k block: half q / 8, chunk q % 8, swizzled by row
-                    const int q = 4 * c + u;
-                    uint32_t o[4];
-                    i4_widen(ws[u], o);
-                    *reinterpret_cast<uint4*>(dst + (q >> 3) * (kI4ABytes / 2) + (((q & 7) ^ (row & 7)) << 4)) =
-                        make_uint4(o[0], o[1], o[2], o[3]);
-                }
+            for (int c2 = 0; c2 < 2; ++c2) {
+                const int c = 4 * h + 2 * part + c2;  // 16-byte chunk of the row (128-byte swizzle)
+                const uint4 w = *reinterpret_cast<const uint4*>(src + ((c ^ (row & 7)) << 4));
+                i4_widen(w.x, &v[16 * c2 + 0]);
+                i4_widen(w.y, &v[16 * c2 + 4]);
+                i4_widen(w.z, &v[16 * c2 + 8]);
+                i4_widen(w.w, &v[16 * c2 + 12]);
             }
-            fence_proxy_async_smem();  // the MMA reads A through the async proxy
+            tmem_st32(tmem_base + lane_addr + kI4AColBase + 64u * (uint32_t)a + 32u * (uint32_t)part, v);
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&afull[a]);
@@ -310,10 +317,10 @@ __global__ void __launch_bounds__(kI4Threads, 1)
             }
         }
     } else {
-        // ------------------------------------------------ accumulate (warps 6-9)
+        // ------------------------------------------------ accumulate (warps 10-13)
         pdl_wait();      // X and Y belong to earlier work on the stream
         cluster_wait();  // every peer's barriers are initialised before the first store into it
-        if (warp == 6 && elect_one()) {
+        if (warp == 2 + kI4WidenWarps && elect_one()) {
             // X (this CTA's K range, all M rows; rows past M and k past K read as 0)
             const int kx0 = kb_lo * kI4BoxK;
             mbar_arrive_expect_tx(xfull, (uint32_t)nxb * xbox_bytes);
@@ -338,13 +345,13 @@ __global__ void __launch_bounds__(kI4Threads, 1)
             const int g = min((kb_lo * kI4BoxK + (i % nblk) * 128) / G, ng - 1);
             return n < N ? __ldg(p.absmax + (size_t)n * ng + g) : 0.0f;
         };
-        // constants of the next 4 blocks load while the current 4 are drained
-        constexpr int kAhead = 4;
+        // constants of the next batch load while the current one is drained
+        constexpr int kAhead = kI4DBatch;
         float a_next[kAhead];
 #pragma unroll
         for (int u = 0; u < kAhead; ++u) a_next[u] = absmax_of(u);
         bool ok = nb > 0;
-        for (int i0 = 0; ok && i0 < nb; i0 += kAhead) {
+        for (int i0 = 0; ok && i0 < nb; i0 += kI4DBatch) {
             float a_cur[kAhead];
 #pragma unroll
             for (int u = 0; u < kAhead; ++u) a_cur[u] = a_next[u];
@@ -352,23 +359,31 @@ __global__ void __launch_bounds__(kI4Threads, 1)
 #pragma unroll
                 for (int u = 0; u < kAhead; ++u) a_next[u] = absmax_of(i0 + kAhead + u);
             }
+            // the commit of the batch's last block completes after every
+            // earlier MMA of the issuing thread, so one wait covers the batch;
+            // the batch's slots are consecutive (i0 is a multiple of 4)
+            const int last = min(i0 + kI4DBatch, nb) - 1;
+            ok = __all_sync(0xffffffffu,
+                            wait_bounded_sleep(&dfull[last % kI4DSlots], (uint32_t)((last / kI4DSlots) & 1), wctx));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t d0 = (uint32_t)(i0 % kI4DSlots);
+            uint32_t r[2][32];
+            tmem_ld32(tmem_base + lane_addr + kI4DColBase + 16u * d0, r[0]);
+            tmem_ld32(tmem_base + lane_addr + kI4DColBase + 16u * d0 + 32u, r[1]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                for (int i = i0; i <= last; ++i) mbar_arrive(&dfree[i % kI4DSlots]);
 #pragma unroll
-            for (int u = 0; u < kAhead; ++u) {
+            for (int u = 0; u < kI4DBatch; ++u) {
                 const int i = i0 + u;
-                if (i >= nb) break;
-                const int j = i / nblk, b = i % nblk, d = i % kI4DSlots;
-                ok = __all_sync(0xffffffffu, wait_bounded_sleep(&dfull[d], (uint32_t)((i / kI4DSlots) & 1), wctx));
-                if (!ok) break;
-                tc_fence_after();
-                uint32_t r[16];
-                tmem_ld16(tmem_base + lane_addr + kI4DColBase + 16u * (uint32_t)d, r);
-                tmem_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&dfree[d]);
+                if (i > last) break;
+                const int j = i / nblk, b = i % nblk;
                 const float sc = __fdiv_rn(a_cur[u], 7.0f);
 #pragma unroll
-                for (int m = 0; m < 16; ++m) y[m] = fmaf(__uint_as_float(r[m]), sc, y[m]);
+                for (int m = 0; m < 16; ++m) y[m] = fmaf(__uint_as_float(r[u >> 1][16 * (u & 1) + m]), sc, y[m]);
                 if (b == nblk - 1) {
                     // tile j is complete in this K range: keep it (owner) or send it to its owner
                     if (j == rank) {
@@ -408,7 +423,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         }
     }
 
-    if (warp < 6) cluster_wait();  // warps 6-9 waited before their first peer access
+    if (warp < 2 + kI4WidenWarps) cluster_wait();  // warps 10-13 waited before their first peer access
     // every store into this CTA's shared memory completes on a barrier it has
     // waited for; after a timeout a peer's store may still be on its way
     if (*abort_flag) settle_after_abort();

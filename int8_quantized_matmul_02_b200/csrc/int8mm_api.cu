@@ -475,44 +475,36 @@ bool int4_shape_ok(int K, int N, int G) {
 
 // Plan of the 4-bit kernel: clusters of `cluster` CTAs split K in 256-k
 // boxes, tiles shared out evenly (at most `cluster` per cluster), one CTA per
-// SM (its shared memory), one wave when the tiles allow.
+// SM (the kernel takes the whole TMEM), one wave when the tiles allow.
 struct Int4Plan {
-    int cluster, clusters, stages, xrows, grid, aslots;
-    uint32_t tmem_cols, off_a, off_x, off_red, off_bars, bytes;
+    int cluster, clusters, stages, xrows, grid;
+    uint32_t tmem_cols, off_x, off_red, off_bars, bytes;
 };
 
-// The first fit in this order: clusters of 4, then 8 CTAs (more CTAs share
-// the K range, so less of X per CTA); three A operands, then two; the most
-// ring stages up to 12 (at least 3).  The kernel keeps its K range of X in
-// shared memory, so K is bounded: with 8-row X boxes (M <= 8) up to about
-// 40 K, with 16-row boxes (M <= 16) up to about 12 K.
 bool int4_plan(int M, int K, int N, DeviceInfo* dev, Int4Plan* P) {
     if (M < 1 || M > kInt4MaxRows) return false;
     const int kbt = cdiv(K, kI4BoxK);
     const int tiles = cdiv(N, kI4TileN);
     const int xrows = M <= 8 ? 8 : 16;
-    const size_t cap = (size_t)kMaxSmemOptin;
-    for (int c : {4, 8}) {
-        const int cl = std::min(c, kbt);
-        int ncl = std::max(1, std::min(tiles, cluster_capacity(dev, cl)));
-        if (cdiv(tiles, ncl) > cl) ncl = cdiv(tiles, cl);
-        const size_t xb = (size_t)cdiv(kbt, cl) * (kI4BoxK / 64) * xrows * 128 + 1024;  // + the row-8 overhang
-        const size_t red = (size_t)cl * kI4TileN * xrows * 4;  // a slot per peer and one for its own sums
-        for (int as = kI4ASlots; as >= 2; --as) {
+    // one CTA per SM (the kernel takes the whole TMEM)
+    for (size_t cap : {(size_t)kMaxSmemOptin}) {
+        for (int c : {4, 8}) {
+            const int cl = std::min(c, kbt);
+            int ncl = std::max(1, std::min(tiles, cluster_capacity(dev, cl)));
+            if (cdiv(tiles, ncl) > cl) ncl = cdiv(tiles, cl);
+            const size_t xb = (size_t)cdiv(kbt, cl) * (kI4BoxK / 64) * xrows * 128 + 1024;  // + the row-8 overhang
+            const size_t red = (size_t)cl * kI4TileN * xrows * 4;  // a slot per peer and one for its own sums
             for (int s = 12; s >= 3; --s) {
                 const size_t bars = (size_t)(2 * s + 2 * kI4ASlots + 2 * kI4DSlots + 3) * 8 + 64;
-                const size_t total = 1024 + (size_t)s * kI4StageBytes + (size_t)as * kI4ABytes + xb + red + bars;
+                const size_t total = 1024 + (size_t)s * kI4StageBytes + xb + red + bars;
                 if (total > cap) continue;
                 P->cluster = cl;
                 P->clusters = ncl;
                 P->stages = s;
                 P->xrows = xrows;
                 P->grid = cl * ncl;
-                P->aslots = as;
                 P->tmem_cols = kI4TmemCols;
                 size_t o = (size_t)s * kI4StageBytes;
-                P->off_a = (uint32_t)o;
-                o += (size_t)as * kI4ABytes;
                 P->off_x = (uint32_t)o;
                 o += xb;
                 P->off_red = (uint32_t)o;
@@ -1148,8 +1140,6 @@ int8mm_status int8mm_forward_int4(const uint16_t* X, int M, const int8mm_int4_we
     p.stages = pl.stages;
     p.xrows = pl.xrows;
     p.tmem_cols = pl.tmem_cols;
-    p.aslots = pl.aslots;
-    p.off_a = pl.off_a;
     p.off_x = pl.off_x;
     p.off_red = pl.off_red;
     p.off_bars = pl.off_bars;

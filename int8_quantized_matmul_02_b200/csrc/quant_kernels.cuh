@@ -150,17 +150,15 @@ __device__ __noinline__ void detect_finalise(const uint32_t* __restrict__ part, 
         const int w = base + tid;
         uint32_t word = 0u;
         if (w < nw) {
-            // eight independent loads in flight per step: the splits' words
-            // come from L2, and this block's latency is on the critical path
-            int y = 0;
-            for (; y + 8 <= ny; y += 8) {
-                uint32_t t[8];
+            // up to 16 independent loads in flight per step (all of them for
+            // up to 16 row splits): this block's latency is on the critical path
+            for (int y0 = 0; y0 < ny; y0 += 16) {
+                uint32_t t[16];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) t[i] = __ldcg(part + (size_t)(y + i) * nw + w);
+                for (int i = 0; i < 16; ++i) t[i] = y0 + i < ny ? __ldcg(part + (size_t)(y0 + i) * nw + w) : 0u;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) word |= t[i];
+                for (int i = 0; i < 16; ++i) word |= t[i];
             }
-            for (; y < ny; ++y) word |= __ldcg(part + (size_t)y * nw + w);
         }
         const int c = __popc(word);
         int incl = c;
@@ -205,7 +203,7 @@ __device__ __noinline__ void detect_finalise(const uint32_t* __restrict__ part, 
 // row splits into the bitmask mask[w], forms the exclusive prefix counts
 // spre[w] (outlier columns before word w) and writes the ascending outlier
 // list idx, the count *n_out and the overflow flag, then resets the ticket.
-__global__ void __launch_bounds__(256) k_detect(const uint16_t* __restrict__ X, int M, int K, float thr,
+__global__ void __launch_bounds__(256, 6) k_detect(const uint16_t* __restrict__ X, int M, int K, float thr,
                                                 int rows_per_block, uint32_t* __restrict__ part,
                                                 uint32_t* __restrict__ mask, int32_t* __restrict__ spre,
                                                 int32_t* __restrict__ idx, int32_t* __restrict__ n_out, int cap,

@@ -43,8 +43,8 @@ def _check_weight(w, W, G):
     (9, 1152, 400, 128),       # K % 256 == 128: the last half box lies past K
     (5, 128, 16, 128),         # one 128-k block, a tile of 16 columns
     (8, 11008, 4096, 128),     # FFN down-projection shape, clusters over 43 boxes
-    (16, 12288, 272, 256),     # the longest K for 16 rows (clusters of 8, two A operands)
-    (8, 40960, 144, 1024),     # the longest K for 8 rows
+    (16, 28672, 144, 256),     # the longest K for 16 rows (clusters of 8, 3 ring stages)
+    (8, 73728, 48, 1024),      # the longest K for 8 rows
 ])
 def test_int4_matches_oracle(cuda_ok, M, K, N, G):
     X, W = _inputs(M, K, N, seed=M * 1000 + K + N + G)
@@ -86,8 +86,8 @@ def test_int4_rejects_bad_shapes(cuda_ok):
     w = i8.prepare_weight_int4(W, 128)
     with pytest.raises(i8.Int8mmError):
         i8.forward_int4(torch.zeros(17, 256, dtype=torch.float16, device="cuda"), w)  # M > 16
-    W2 = torch.zeros(12416, 16, dtype=torch.float16, device="cuda")
+    W2 = torch.zeros(28928, 16, dtype=torch.float16, device="cuda")
     w2 = i8.prepare_weight_int4(W2, 128)
-    i8.forward_int4(torch.zeros(8, 12416, dtype=torch.float16, device="cuda"), w2)  # fits with 8 rows
+    i8.forward_int4(torch.zeros(8, 28928, dtype=torch.float16, device="cuda"), w2)  # fits with 8 rows
     with pytest.raises(i8.Int8mmError):
-        i8.forward_int4(torch.zeros(9, 12416, dtype=torch.float16, device="cuda"), w2)  # X share too long
+        i8.forward_int4(torch.zeros(9, 28928, dtype=torch.float16, device="cuda"), w2)  # X share too long
