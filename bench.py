@@ -9,7 +9,7 @@ throughput in int8 TOPS (2*M*N*K per forward, all K counted) with the
 dominant kernel's roofline against the dense-int8 tensor peak.  Objects on the
 same line:
   decode       the decode-shaped FFN up-projection (X 8 x 4096, W 4096 x 11008)
-               in HBM GB/s against the measured copy bandwidth, judged on
+               in HBM GB/s against the measured copy bandwidth, measured on
                forwards back to back (the launch alone reported beside it);
   configs      the prefill FFN and the attention-QKV sweep (0, 12, 48, 123
                outlier columns and threshold = inf) in TOPS;
@@ -763,7 +763,7 @@ def main():
                 "value": step_gbs, "us_per_step": d["plain_us"], "graph_us_per_step": d["graph_us"],
                 "graph_value": d["bytes"] / (d["graph_us"] * 1e-6) / 1e9,
                 "algorithmic_bytes": d["bytes"], "outlier_columns_detected": d["n_o"],
-                # the target is judged on the step: forwards back to back, each
+                # the roofline fraction is the step's: forwards back to back, each
                 # launched while the previous one finishes (as in a model's
                 # layer sequence); the launch alone is reported beside it
                 "roofline": {"bound": "hbm", "kernel": "k_decode_int8_sm100", "basis": "back-to-back step",
