@@ -2,13 +2,18 @@
 // conversion ("LLM.int8(): 8-bit Matrix Multiplication for Transformers at
 // Scale", abstract):
 //   k_col_absmax / k_quant_weight   -- per-output-channel absmax int8 weight (c)
-//   k_detect                        -- outlier feature columns of X (a)
-//   k_quant_rows                    -- row absmax int8 X without the outlier
-//                                      columns, plus the fp16 outlier columns (b)
+//   k_detect                        -- outlier feature columns of X, their
+//                                      list and count (a)
+//   k_quant_rows_reg (K <= 16384) /
+//   k_quant_rows (longer K)         -- row absmax int8 X without the outlier
+//                                      columns, plus the fp16 outlier columns (b);
+//                                      the first also gathers the outlier
+//                                      weight rows in the same grid
 //   k_col_absmax_grouped /
 //   k_quant_rows_grouped            -- the same with one constant per group of G
 //                                      consecutive k (group-wise variant)
-//   k_gather_wo                     -- fp16 weight rows of the outlier dims (d)
+//   k_gather_wo                     -- fp16 weight rows of the outlier dims (d),
+//                                      for the paths without k_quant_rows_reg
 // All loads of X / W are 16-byte vectors along the contiguous dimension.
 #pragma once
 
