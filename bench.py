@@ -21,7 +21,10 @@ same line:
 One step = one whole forward (outlier detection, X quantisation, outlier weight
 gather, int8 GEMM with fused dequantising epilogue and fp16 outlier product);
 the weight is prepared once, outside the timed region.  Inputs are synthetic
-and seeded (see int8_quantized_matmul_02_b200.synth).
+and seeded (see int8_quantized_matmul_02_b200.synth).  The `e2e` key is the
+same metric through the public call with host buffers (int8mm_forward_host:
+pinned X copied in, Y copied back to pinned memory in row bands that overlap
+the product), the copies inside the timed region.
 
 Multi-GPU: the path is one GPU with no collective; --gpus N runs N
 independent replicas (one process per GPU, torchrun), weak scaling, timed as
@@ -314,8 +317,10 @@ def run_gemm_workload(wl, steps: int, warmup: int, dev, rank: int, cap: int):
 
 
 def run_e2e(wl, state, steps: int, dev):
-    """Same metric through the public API with host buffers: pinned X in,
-    fp16 Y out, both copies inside the timed region."""
+    """Same metric through the public API with host buffers (the package's
+    forward() with a pinned CPU X and a pinned CPU Y, which calls
+    int8mm_forward_host): X copied in, Y copied back in row bands overlapping
+    the product, every copy inside the timed region."""
     import int8_quantized_matmul_02_b200 as i8
 
     Xh = state["X"].pin_memory()
