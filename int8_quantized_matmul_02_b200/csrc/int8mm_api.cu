@@ -943,8 +943,12 @@ int8mm_status int8mm_forward_host(const uint16_t* x_host, int M, const int8mm_we
                                   int max_outliers, uint16_t* y_host, uint16_t* x_dev, uint16_t* y_dev,
                                   void* ws, size_t ws_bytes, void* stream) {
     if (!x_host || !y_host || !x_dev || !y_dev || !w) return INT8MM_ERR_INVALID_ARGUMENT;
-    const int K = w->K, N = w->N;
-    if (!shape_ok(M, K, N)) return INT8MM_ERR_INVALID_ARGUMENT;
+    const int K = w->K;
+    // argument errors first, before the device is touched or anything is queued
+    {
+        const int8mm_status chk = forward_check(x_dev, M, w, threshold, max_outliers, y_dev, ws, ws_bytes);
+        if (chk != INT8MM_OK) return chk;
+    }
     int dev;
     DeviceInfo* info;
     int8mm_status st = current_device(&dev, &info);
@@ -963,11 +967,6 @@ int8mm_status int8mm_forward_host(const uint16_t* x_host, int M, const int8mm_we
         hp.ready = true;
     }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // argument errors first, before anything is queued
-    {
-        const int8mm_status chk = forward_check(x_dev, M, w, threshold, max_outliers, y_dev, ws, ws_bytes);
-        if (chk != INT8MM_OK) return chk;
-    }
     cudaError_t e = cudaMemcpyAsync(x_dev, x_host, (size_t)M * K * 2, cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) return cuda_status(e);
     HostCopy hc{y_host, hp.copy, hp.band_done, hp.copies_done, kHostBands};

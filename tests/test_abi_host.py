@@ -96,6 +96,31 @@ def test_forward_rejects_bad_arguments(lib):
     assert _fwd(lib, opts=_abi.ForwardOpts(7, None, 0)) == 1
 
 
+def _fwd_host(lib, Xh=FAKE, M=16, w=None, thr=6.0, cap=0, Yh=FAKE, Xd=FAKE, Yd=FAKE, ws=FAKE, nbytes=1 << 30):
+    w = w or _weight()
+    return lib.int8mm_forward_host(ctypes.c_void_p(Xh), M, ctypes.byref(w), thr, cap, ctypes.c_void_p(Yh),
+                                   ctypes.c_void_p(Xd), ctypes.c_void_p(Yd), ctypes.c_void_p(ws), nbytes, None)
+
+
+def test_host_forward_rejects_bad_arguments_before_the_device(lib):
+    """int8mm_forward_host checks every argument before it touches the
+    device (so these calls return the same codes on a machine without one)."""
+    assert _fwd_host(lib, Xh=0) == 1
+    assert _fwd_host(lib, Yh=0) == 1
+    assert _fwd_host(lib, Xd=0) == 1
+    assert _fwd_host(lib, Yd=0) == 1
+    assert _fwd_host(lib, ws=0) == 1
+    assert _fwd_host(lib, M=0) == 1
+    assert _fwd_host(lib, thr=float("nan")) == 1
+    assert _fwd_host(lib, cap=257) == 1
+    assert _fwd_host(lib, w=_weight(K=250)) == 1
+    assert _fwd_host(lib, Xd=FAKE + 2) == 2       # device staging buffers: 16-byte aligned
+    assert _fwd_host(lib, Yd=FAKE + 8) == 2
+    assert _fwd_host(lib, ws=FAKE + 16) == 2
+    need = lib.int8mm_workspace_bytes(16, 256, 384, 0)
+    assert _fwd_host(lib, nbytes=need - 1) == 3
+
+
 def test_forward_rejects_misaligned_pointers(lib):
     assert _fwd(lib, X=FAKE + 2) == 2
     assert _fwd(lib, Y=FAKE + 8) == 2
